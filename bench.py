@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of paged absorbed-MLA decode (plan + split scan + combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the split planner, the
+split scan (the dominant kernel) and the LSE combine, on inputs already resident in HBM.
+Prints ONE JSON line on rank 0.  value = KV-read GB/s of the whole job (bytes of cache
+rows the decode must read, summed over ranks, divided by the slowest rank's device
+time); us_per_call is the per-step latency.  The L2 (126 MB) is flushed by a 256 MB
+write between timed steps, outside the timed events.
+
+Multi-GPU (torchrun): every rank decodes its own replica of the workload (requests are
+independent; there is no data-path collective), time = max over ranks, scaling weak.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the same workload
+and reports it in the same metric, extrapolated by rows (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from mla_attention_decode_paged_b200 import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "agent_spec"
+METRIC = "MLA decode KV-read GB/s (us/call; % of B200 HBM/tensor roofline)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_simt.cu"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the scan kernel from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def workload_desc(wl):
+    s = wl.spec
+    lens = wl.seq_lens
+    return (f"{s.name}: B={s.B} s_q={s.s_q} H={s.H} (M={s.M}) T={int(lens.min())}..{int(lens.max())} "
+            f"(sum {int(lens.sum())}) page=64 {'e4m3' if s.kv_dtype else 'bf16'} KV, "
+            f"{'causal' if s.causal else 'non-causal'}, shuffled block_table, seed {s.seed}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while alive."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(wl, n_req=None):
+    """Time the oracle on n_req requests x a head subset giving 16 rows (one oracle row
+    block) per request; returns (seconds for the full workload, extrapolated by rows and
+    by the sampled requests' share of cache tokens, threads used, description)."""
+    import oracle
+    heads = list(range(max(1, min(wl.H, 16 // wl.s_q))))
+    reqs = list(range(wl.B if n_req is None else max(1, min(wl.B, n_req))))
+    rows_s = wl.s_q * len(heads)
+    t0 = time.perf_counter()
+    oracle.mla_decode(wl.q[reqs][:, :, heads], wl.kv, wl.kv_dtype, wl.kv_scale, wl.block_table[reqs],
+                      wl.seq_lens[reqs], wl.scale, wl.causal)
+    dt = time.perf_counter() - t0
+    tok_share = float(wl.seq_lens[reqs].astype(np.int64).sum()) / float(wl.seq_lens.astype(np.int64).sum())
+    full = dt * (wl.spec.M / rows_s) / tok_share
+    cores = min(len(reqs) * ((rows_s + 15) // 16), len(os.sched_getaffinity(0)))
+    desc = (f"oracle on {len(reqs)} of {wl.B} requests x {len(heads)} head(s) x {wl.s_q} drafts = {rows_s} of "
+            f"{wl.spec.M} rows per request ({dt:.2f} s), scaled by rows and cache tokens to the full workload")
+    return full, cores, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.make_workload(args.workload)
+    kvb = wl.kv_bytes()
+    # size the per-step sample so that the whole run stays within about two minutes
+    n_req = wl.B
+    t0 = time.perf_counter()
+    oracle_sample(wl, n_req)
+    first = time.perf_counter() - t0
+    n_steps = args.warmup - 1 + args.steps
+    if first * n_steps > 120.0:
+        n_req = max(1, int(wl.B * 120.0 / (first * n_steps)))
+    for _ in range(args.warmup - 1):
+        oracle_sample(wl, n_req)
+    times = []
+    cores, desc = 0, ""
+    for _ in range(args.steps):
+        t, cores, desc = oracle_sample(wl, n_req)
+        times.append(t)
+    step = sum(times) / len(times)
+    value = kvb / step / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "us_per_call": step * 1e6,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl), "global_batch": wl.B, "seq_len": int(wl.seq_lens.max()),
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mla_attention_decode_paged_b200 as mla
+    from mla_attention_decode_paged_b200 import build as build_mod
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    build_mod.build(quiet=True)
+
+    wl = W.make_workload(args.workload)
+    q, kv, bt, sl = (torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).to(dev),
+                     (torch.from_numpy(wl.kv.view(np.int16)).view(torch.bfloat16) if wl.kv_dtype == W.KV_BF16
+                      else torch.from_numpy(wl.kv)).to(dev),
+                     torch.from_numpy(wl.block_table).to(dev), torch.from_numpy(wl.seq_lens).to(dev))
+    ws = mla.alloc_workspace(wl.B, wl.s_q, wl.H, device=dev)
+    out = torch.empty((wl.B, wl.s_q, wl.H, W.DV), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.B, wl.s_q, wl.H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mla.plan(sl, wl.s_q, wl.H, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, ws, out, lse, kv_scale=wl.kv_scale, stream=stream,
+                   scan_only=True)
+        if ev is not None:
+            ev[2].record(stream)
+        mla.combine(ws, wl.B, wl.s_q, wl.H, out, lse, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.random_(0, 255)
+        step()
+    torch.cuda.synchronize(dev)
+    assert mla.device_status(ws, stream=stream) == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.random_(0, 255)  # outside the timed events
+            step(evs[k])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    plan_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    scan_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    tot = torch.tensor([sum(step_ms), sum(scan_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    tot_ms, tot_scan_ms = float(tot[0]), float(tot[1])
+
+    # end to end through the same public calls with host buffers: pinned inputs copied in,
+    # outputs copied out, every step.  The cache itself stays resident (it is the state).
+    q_h = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    bt_h = torch.from_numpy(wl.block_table).pin_memory()
+    sl_h = torch.from_numpy(wl.seq_lens).pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    def e2e_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        q.copy_(q_h, non_blocking=True)
+        bt.copy_(bt_h, non_blocking=True)
+        sl.copy_(sl_h, non_blocking=True)
+        mla.plan(sl, wl.s_q, wl.H, ws, stream=stream)
+        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, ws, out, lse, kv_scale=wl.kv_scale, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.random_(0, 255)
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    for k in range(args.steps):
+        flush.random_(0, 255)
+        e2e_step(e2e_ev[k])
+    torch.cuda.synchronize(dev)
+    e2e_tot = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in e2e_ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_tot, op=dist.ReduceOp.MAX)
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    kvb = wl.kv_bytes()
+    flops = wl.flops()
+    value = kvb * world * args.steps / (tot_ms * 1e-3) / 1e9
+    e2e_value = kvb * world * args.steps / (float(e2e_tot[0]) * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    scan_avg_s = tot_scan_ms * 1e-3 / args.steps
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    intensity = flops / kvb
+    if intensity < ridge:
+        roof = {"bound": "hbm", "achieved": kvb / scan_avg_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / scan_avg_s / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe'})"
+    roof["kernel"] = "mla decode split scan"
+    roof["traffic"] = ncu_traffic(args.workload)
+    roof["algorithmic_bytes_per_launch"] = kvb
+    roof["algorithmic_flops_per_launch"] = flops
+    t_roof = max(kvb / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "us_per_call": tot_ms / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.kv_dtype == W.KV_BF16 else "e4m3->bf16",
+            "data": "synthetic (seeded N(0,1) q/KV; no dataset)",
+            "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": int(wl.seq_lens.max()),
+                       "parallelism": f"replicas x{world} (no collective)",
+                       "l2": "flushed between steps by a 256 MB write outside the timed events"},
+            "breakdown_us": {"plan": statistics.median(plan_ms) * 1e3, "scan": statistics.median(scan_ms) * 1e3,
+                             "combine": statistics.median(comb_ms) * 1e3},
+            "tflops": flops * world * args.steps / (tot_ms * 1e-3) / 1e12,
+            "roofline_us": t_roof * 1e6, "frac_of_roofline_step": t_roof / (tot_ms * 1e-3 / args.steps),
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "us_per_call": float(e2e_tot[0]) / args.steps * 1e3,
+                    "note": "q, block_table, seq_lens in and out, lse out per step; the paged cache stays resident"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        full_s, cores, desc = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": kvb / full_s / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warmup raised to 3 (minimum)")
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

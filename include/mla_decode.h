@@ -1,0 +1,148 @@
+/*
+ * mla_decode.h -- C ABI of the paged, weight-absorbed MLA decode library
+ * (libmla_decode.so, CUDA for sm_100a).
+ *
+ * The operation.  Multi-head Latent Attention keeps one shared latent row per cached
+ * token: a 512-wide c_kv plus a decoupled 64-wide RoPE key, 576 values in all
+ * ["TokenSpeed" related-work notes (zhaifeiyue.github.io), DeepSeek-V3 entry: 512-dim
+ * latent KV; llm-atlas "Inference systems", 22 DeepSeek V2->V3: RoPE part decoupled].
+ * Decode runs in that latent space ("absorb + project", same entry): the caller has
+ * already multiplied the no-RoPE query through W_UK, so q is 576 wide, and multiplies
+ * the 512-wide output through W_UV afterwards.  The s_q speculative query tokens of a
+ * request and its H heads are folded into one row axis of M = s_q * H rows, row
+ * m = i * H + h, all attending to the same cached rows ("TokenSpeed" launch digest
+ * (cvshuo.com), MLA kernel paragraphs: the query-sequence axis is folded into the
+ * head axis to fill the M tile; zhaifeiyue notes, Attack 1: H_eff = num_heads x F).
+ * The cache is paged: logical block p of request b lives in physical page
+ * block_table[b][p] [llm-atlas "Inference systems", 07 PagedAttention].  Draft token
+ * i of request b sees cached tokens t <= T_b - s_q + i (causal) or t < T_b, i.e.
+ * seq_lens counts the drafts, whose rows are the last s_q rows of the cache
+ * [llm-atlas "Inference systems", 16 Speculative decoding: candidates verified in
+ * parallel].  For each row:
+ *     s_t = scale * q . KV_t,   out = sum_t softmax(s)_t * KV_t[0:512],
+ *     lse = ln sum_t exp(s_t).
+ * Long caches are scanned in splits whose partial (out, lse) are merged by an
+ * LSE-weighted combine ["Faster kernels, slower engine" (jinnpan.com), 7.1 Gluon MLA
+ * decode: split-KV scan and reduction].  An fp8 cache stores e4m3 bytes with one
+ * fp32 scale per tensor, value = e4m3(byte) * kv_scale ["Faster kernels, slower
+ * engine", setup note on the fp8 KV cache: half the bytes per cached token].
+ *
+ * Conventions for every entry point.
+ *  - Pointers are DEVICE pointers unless marked host.  All arrays are dense,
+ *    row-major, and start on a 16-byte boundary (the cache and q on 128 bytes).
+ *  - The caller owns every buffer, including the workspace; nothing is retained after
+ *    a call returns.  mla_decode_plan / mla_decode / mla_split_kv_combine never
+ *    allocate, free or synchronise: they enqueue work on `stream` (a cudaStream_t,
+ *    0 = legacy default stream) and return.
+ *  - Errors are return codes; nothing is thrown across the ABI.  Arguments are
+ *    checked on the host before anything is enqueued.  Conditions only the device can
+ *    see (a page id outside [0, num_pages), seq_len outside [1, max_pages * 64], or
+ *    seq_len < s_q under the causal rule) set a status word in the workspace and turn
+ *    the affected rows into NaN; read it with mla_get_device_status.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,         /* null pointer, non-positive size, non-finite scale */
+    MLA_ERR_UNSUPPORTED = 2,         /* shape or dtype the kernels do not handle */
+    MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < mla_decode_workspace_size(...) */
+    MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+    MLA_ERR_DEVICE_OOB = 5,          /* device status: bad page id or sequence length */
+    MLA_ERR_DEVICE_TIMEOUT = 6,      /* device status: a bounded wait gave up */
+    MLA_ERR_PLAN_MISMATCH = 7        /* device status: workspace plan made for other B/s_q/H */
+} mla_status;
+
+typedef enum { MLA_KV_BF16 = 0, MLA_KV_E4M3 = 1 } mla_kv_dtype;
+
+/* Fixed geometry of the latent row and the page. */
+#define MLA_HEAD_DIM_QK 576
+#define MLA_HEAD_DIM_V 512
+#define MLA_PAGE_SIZE 64
+
+/*
+ * Bytes of workspace a plan + decode of this shape needs (host, pure).
+ * num_sms: SM count the split plan is made for; 0 = the current device's.
+ * Returns 0 for an unsupported shape (B, s_q, H <= 0, or s_q * H > 65536).
+ */
+size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
+
+/*
+ * Split planner (one small kernel on `stream`).  From seq_lens[B] (device int32) it
+ * partitions the pages of all requests into equal contiguous shares, one share per
+ * group of SM pairs, cutting requests into splits where a share ends.  The plan is
+ * written into `workspace` and is valid for every later mla_decode of the same
+ * seq_lens, B, s_q and H (e.g. all layers of one decode step).  num_sms as above; a
+ * smaller value gives fewer, longer splits (2 = no splits at all).
+ */
+mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, int H, int num_sms,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Paged absorbed-MLA decode: split scan over the plan in `workspace`, then the
+ * split-KV combine.
+ *   q           bf16 [B, s_q, H, 576]
+ *   kv_pages    bf16 or e4m3 [num_pages, 64, 576]
+ *   kv_dtype    MLA_KV_BF16 or MLA_KV_E4M3; kv_scale multiplies e4m3 values (ignored
+ *               for bf16; must be finite and > 0 for e4m3)
+ *   block_table int32 [B, max_pages_per_req]; entries past ceil(T_b / 64) are never
+ *               read
+ *   seq_lens    int32 [B], T_b >= 1, T_b <= max_pages_per_req * 64, and T_b >= s_q
+ *               when causal != 0 (the same array the plan was made from)
+ *   scale       softmax scale applied to the full 576-wide dot product
+ *   causal      != 0: draft i sees t <= T_b - s_q + i; 0: every t < T_b
+ *   out         bf16 [B, s_q, H, 512];  lse  fp32 [B, s_q, H], natural log
+ * Supported: s_q * H <= 256 per request.
+ */
+mla_status mla_decode(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,
+                      const int32_t* block_table, int max_pages_per_req,
+                      const int32_t* seq_lens, int B, int s_q, int H, int64_t num_pages,
+                      float scale, int causal, void* workspace, size_t ws_bytes, void* out,
+                      float* lse, void* stream);
+
+/*
+ * The split scan of mla_decode alone (same arguments): rows of unsplit requests get
+ * their final out / lse, split requests leave per-split partials in `workspace` for
+ * mla_split_kv_combine.  mla_decode == mla_decode_scan followed by
+ * mla_split_kv_combine; the two halves are exported so that each can be run and timed
+ * on its own.
+ */
+mla_status mla_decode_scan(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,
+                           const int32_t* block_table, int max_pages_per_req,
+                           const int32_t* seq_lens, int B, int s_q, int H, int64_t num_pages,
+                           float scale, int causal, void* workspace, size_t ws_bytes, void* out,
+                           float* lse, void* stream);
+
+/*
+ * The LSE-weighted combine of the split partials held in `workspace`: for every row of
+ * a request that the plan split, lse = ln sum_j exp(lse_j) and
+ * out = sum_j exp(lse_j - lse) * out_j (bf16); empty splits (lse_j = -inf) drop out.
+ * Rows of unsplit requests are left untouched.  mla_decode calls it; it is exported so
+ * that it can be run (and timed) on its own.
+ */
+mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, int s_q, int H,
+                                void* out, float* lse, void* stream);
+
+/*
+ * Reads and clears the device status word of `workspace` (host out: *code, one of
+ * MLA_OK, MLA_ERR_DEVICE_OOB, MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_PLAN_MISMATCH).  This
+ * call synchronises `stream`; it is meant for tests and debugging.
+ */
+mla_status mla_get_device_status(void* workspace, int* code, void* stream);
+
+/* Library version string (host, static storage). */
+const char* mla_decode_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

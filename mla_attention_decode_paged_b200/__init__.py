@@ -1,0 +1,90 @@
+"""Paged, weight-absorbed MLA decode for B200 (sm_100a).
+
+The work happens in ``libmla_decode.so`` (C ABI declared in ``include/mla_decode.h``);
+``_abi`` binds its entry points under the same names, and the helpers below only turn
+torch CUDA tensors into pointers and sizes.  torch is used for device memory and
+streams, nothing else.
+"""
+from __future__ import annotations
+
+from . import _abi
+from ._abi import (MLA_KV_BF16, MLA_KV_E4M3, MlaError, mla_decode_plan, mla_decode_version,
+                   mla_decode_workspace_size, mla_get_device_status, mla_split_kv_combine)
+
+PAGE = 64
+DQK = 576
+DV = 512
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise MlaError(rc, what)
+
+
+def workspace_bytes(B: int, s_q: int, H: int, num_sms: int = 0) -> int:
+    n = mla_decode_workspace_size(B, s_q, H, num_sms)
+    if n == 0:
+        raise MlaError(_abi.MLA_ERR_UNSUPPORTED, "mla_decode_workspace_size")
+    return n
+
+
+def alloc_workspace(B: int, s_q: int, H: int, num_sms: int = 0, device=None):
+    """A uint8 CUDA tensor large enough (and 256-byte aligned) for plan + decode."""
+    import torch
+    n = workspace_bytes(B, s_q, H, num_sms)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def plan(seq_lens, s_q: int, H: int, workspace, num_sms: int = 0, stream=None):
+    """Enqueue the split planner for int32 CUDA ``seq_lens`` [B] into ``workspace``."""
+    B = int(seq_lens.shape[0])
+    _check(mla_decode_plan(seq_lens.data_ptr(), B, s_q, H, num_sms, workspace.data_ptr(), workspace.numel(),
+                           _stream_ptr(stream)), "mla_decode_plan")
+
+
+def decode(q, kv_pages, block_table, seq_lens, scale: float, causal: bool, workspace, out, lse,
+           kv_scale: float = 1.0, stream=None, scan_only: bool = False):
+    """Enqueue mla_decode (decode + split combine) on torch CUDA tensors.
+
+    q bf16 [B, s_q, H, 576]; kv_pages bf16 or uint8 (e4m3 bytes) / float8_e4m3fn
+    [P, 64, 576]; block_table int32 [B, max_pages]; seq_lens int32 [B]; out bf16
+    [B, s_q, H, 512]; lse float32 [B, s_q, H].  The plan in ``workspace`` must have
+    been made from the same seq_lens.  ``scan_only`` runs the split scan without the
+    combine (mla_decode_scan); follow it with ``combine``.
+    """
+    import torch
+    B, s_q, H, d = q.shape
+    assert d == DQK and q.dtype == torch.bfloat16 and q.is_contiguous()
+    if kv_pages.dtype == torch.bfloat16:
+        kv_dtype = MLA_KV_BF16
+    elif kv_pages.dtype in (torch.uint8, torch.float8_e4m3fn):
+        kv_dtype = MLA_KV_E4M3
+    else:
+        raise TypeError(f"unsupported cache dtype {kv_pages.dtype}")
+    assert kv_pages.is_contiguous() and kv_pages.shape[1:] == (PAGE, DQK)
+    assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+    assert seq_lens.dtype == torch.int32 and out.dtype == torch.bfloat16 and lse.dtype == torch.float32
+    fn = _abi.mla_decode_scan if scan_only else _abi.mla_decode
+    _check(fn(q.data_ptr(), kv_pages.data_ptr(), kv_dtype, float(kv_scale), block_table.data_ptr(),
+              int(block_table.shape[1]), seq_lens.data_ptr(), B, s_q, H, int(kv_pages.shape[0]),
+              float(scale), int(bool(causal)), workspace.data_ptr(), workspace.numel(),
+              out.data_ptr(), lse.data_ptr(), _stream_ptr(stream)), "mla_decode_scan" if scan_only else "mla_decode")
+
+
+def combine(workspace, B: int, s_q: int, H: int, out, lse, stream=None):
+    _check(mla_split_kv_combine(workspace.data_ptr(), workspace.numel(), B, s_q, H, out.data_ptr(),
+                                lse.data_ptr(), _stream_ptr(stream)), "mla_split_kv_combine")
+
+
+def device_status(workspace, stream=None) -> int:
+    """Read and clear the device status word (synchronises the stream)."""
+    rc, code = mla_get_device_status(workspace.data_ptr(), _stream_ptr(stream))
+    _check(rc, "mla_get_device_status")
+    return code

@@ -1,0 +1,30 @@
+// mla_decode_params.cuh -- argument block passed from the host entry point to the
+// decode kernels.
+#pragma once
+
+#include "mla_common.cuh"
+
+namespace mla {
+
+struct DecodeParams {
+    const void* q;              // bf16 [B, s_q, H, 576]
+    const void* kv;             // bf16 / e4m3 [num_pages, 64, 576]
+    const int32_t* block_table; // [B, max_pages]
+    const int32_t* seq_lens;    // [B]
+    void* ws;                   // workspace (plan + partials)
+    void* out;                  // bf16 [B, s_q, H, 512]
+    float* lse;                 // fp32 [B, s_q, H]
+    int64_t num_pages;
+    int max_pages;
+    int B, s_q, H, M;
+    int causal;
+    int groups_launched;        // groups the grid covers (>= the plan's)
+    float score_scale_log2;     // scale * kv_scale * log2(e): scores in base 2
+    float out_scale;            // kv_scale for e4m3 (values are e4m3 * kv_scale), 1 for bf16
+};
+
+mla_status launch_decode_simt(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
+mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream);
+int device_sm_count();
+
+}  // namespace mla

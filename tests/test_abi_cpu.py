@@ -1,0 +1,97 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry point, sizes
+workspaces, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_attention_decode_paged_b200 as mla
+from mla_attention_decode_paged_b200 import _abi
+from mla_attention_decode_paged_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_mod.build(quiet=True)
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(mla_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_entry_point():
+    names = declared_functions()
+    assert {"mla_decode", "mla_decode_plan", "mla_split_kv_combine", "mla_decode_workspace_size",
+            "mla_get_device_status"} <= set(names)
+    L = ctypes.CDLL(_abi.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared but not exported"
+
+
+def test_version_string():
+    assert "sm_100a" in mla.mla_decode_version()
+
+
+def test_workspace_size_is_pure_host_and_grows_with_shape():
+    a = mla.mla_decode_workspace_size(4, 4, 16, 148)
+    b = mla.mla_decode_workspace_size(16, 16, 16, 148)
+    assert a > 0 and b > a
+    assert a % 256 == 0
+    # partials: (B + groups) x row blocks x 128 rows x 512 fp32 at least
+    assert b >= (16 + 37) * 2 * 128 * 512 * 4
+    assert mla.mla_decode_workspace_size(0, 4, 16, 148) == 0
+    assert mla.mla_decode_workspace_size(4, -1, 16, 148) == 0
+
+
+def _decode_args(**kw):
+    a = dict(q_ptr=16, kv_ptr=16, kv_dtype=0, kv_scale=1.0, block_table_ptr=16, max_pages_per_req=4,
+             seq_lens_ptr=16, B=2, s_q=4, H=16, num_pages=8, scale=0.07, causal=1, workspace_ptr=256,
+             ws_bytes=1 << 30, out_ptr=16, lse_ptr=16, stream=None)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q_ptr=None), _abi.MLA_ERR_INVALID_ARG),
+    (dict(out_ptr=None), _abi.MLA_ERR_INVALID_ARG),
+    (dict(B=0), _abi.MLA_ERR_INVALID_ARG),
+    (dict(num_pages=0), _abi.MLA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _abi.MLA_ERR_INVALID_ARG),
+    (dict(kv_dtype=3), _abi.MLA_ERR_UNSUPPORTED),
+    (dict(kv_dtype=1, kv_scale=0.0), _abi.MLA_ERR_INVALID_ARG),
+    (dict(kv_dtype=1, kv_scale=float("inf")), _abi.MLA_ERR_INVALID_ARG),
+    (dict(s_q=17, H=16), _abi.MLA_ERR_UNSUPPORTED),
+    (dict(q_ptr=18), _abi.MLA_ERR_INVALID_ARG),
+    (dict(workspace_ptr=272), _abi.MLA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), _abi.MLA_ERR_WORKSPACE_TOO_SMALL),
+])
+def test_decode_rejects_bad_arguments_before_any_launch(kw, code):
+    a = _decode_args(**kw)
+    assert _abi.mla_decode(*a.values()) == code
+
+
+def test_plan_rejects_bad_arguments():
+    assert _abi.mla_decode_plan(None, 2, 4, 16, 148, 256, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_decode_plan(16, 2, 4, 16, 148, 256, 1024, None) == _abi.MLA_ERR_WORKSPACE_TOO_SMALL
+    assert _abi.mla_decode_plan(16, 2, 4, 16, 1, 256, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_decode_plan(16, 2, 4, 16, 148, 300, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
+
+
+def test_combine_rejects_bad_arguments():
+    assert _abi.mla_split_kv_combine(None, 1 << 30, 2, 4, 16, 16, 16, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_split_kv_combine(256, 1 << 30, 2, 32, 16, 16, 16, None) == _abi.MLA_ERR_UNSUPPORTED
+    assert _abi.mla_split_kv_combine(256, 16, 2, 4, 16, 16, 16, None) == _abi.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_status_query_rejects_null():
+    rc, _ = _abi.mla_get_device_status(None, None)
+    assert rc == _abi.MLA_ERR_INVALID_ARG
