@@ -138,6 +138,36 @@ mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, i
  */
 mla_status mla_get_device_status(void* workspace, int* code, void* stream);
 
+/*
+ * mla_decode without a caller-provided workspace, for callers that cannot allocate
+ * device memory: a plugin inside another runtime that owns all device memory and
+ * forbids allocation on its execution path, or a latency-critical path that cannot
+ * afford cudaMalloc's implicit device-wide synchronisation.  (The TokenSpeed pages
+ * have no counterpart of this entry point; it is a property of this library.)
+ *
+ * Same arguments and results as mla_decode minus the workspace; it runs the planner,
+ * the split scan and the combine.  The workspace is a scratch array compiled into the
+ * library, MLA_NOALLOC_SCRATCH_BYTES (48 MiB) of device memory that every GPU which
+ * loads the library holds until the process exits.  Nothing is allocated or freed by
+ * the call.  Shapes whose plan needs more scratch than that return
+ * MLA_ERR_WORKSPACE_TOO_SMALL (use mla_decode with your own workspace instead); the
+ * five reference workloads, up to B = 32 requests of s_q * H = 256 rows, fit.
+ *
+ * The first call on a device looks up the scratch array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * Every call shares the one array and the array keeps the last call's contents: the
+ * planner rewrites everything that a call reads before reading it, but calls whose
+ * work overlaps on the GPU (several streams, or several host threads on one device)
+ * race on the scratch and give wrong results.  Serialise them.  Device-side errors
+ * (bad page id or length) show only as NaN rows here: there is no workspace whose
+ * status word the caller could read.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (48u << 20)
+mla_status mla_decode_noalloc(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,
+                              const int32_t* block_table, int max_pages_per_req,
+                              const int32_t* seq_lens, int B, int s_q, int H, int64_t num_pages,
+                              float scale, int causal, void* out, float* lse, void* stream);
+
 /* Library version string (host, static storage). */
 const char* mla_decode_version(void);
 

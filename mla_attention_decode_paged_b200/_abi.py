@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.restype = I
         L.mla_decode_scan.argtypes = [P, P, I, F, P, I, P, I, I, I, I64, F, I, P, SZ, P, P, P]
         L.mla_decode_scan.restype = I
+        L.mla_decode_noalloc.argtypes = [P, P, I, F, P, I, P, I, I, I, I64, F, I, P, P, P]
+        L.mla_decode_noalloc.restype = I
         L.mla_split_kv_combine.argtypes = [P, SZ, I, I, I, P, P, P]
         L.mla_split_kv_combine.restype = I
         L.mla_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
@@ -82,6 +84,13 @@ def mla_decode_scan(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_page
     return lib().mla_decode_scan(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_pages_per_req, seq_lens_ptr,
                                  B, s_q, H, num_pages, scale, int(causal), workspace_ptr, ws_bytes, out_ptr, lse_ptr,
                                  stream)
+
+
+def mla_decode_noalloc(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_pages_per_req, seq_lens_ptr, B,
+                       s_q, H, num_pages, scale, causal, out_ptr, lse_ptr, stream) -> int:
+    """mla_decode on the library's static scratch (no workspace argument, no allocation)."""
+    return lib().mla_decode_noalloc(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_pages_per_req,
+                                    seq_lens_ptr, B, s_q, H, num_pages, scale, int(causal), out_ptr, lse_ptr, stream)
 
 
 def mla_split_kv_combine(workspace_ptr, ws_bytes, B, s_q, H, out_ptr, lse_ptr, stream) -> int:
