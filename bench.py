@@ -190,6 +190,16 @@ def run_reference(args):
     return 0
 
 
+def soak(step, flush, dev, seconds):
+    import torch
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(10):
+            flush.random_(0, 255)
+            step()
+        torch.cuda.synchronize(dev)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -239,16 +249,21 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     assert mla.device_status(ws, stream=stream) == 0
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
+        # The timed steps take milliseconds, shorter than the sampler's 200 ms period, so
+        # identical untimed steps run for a soak window before and after them; the clock
+        # record covers the soak and the timed steps together.
+        soak(step, flush, dev, args.soak_s)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         for k in range(args.steps):
             flush.random_(0, 255)  # outside the timed events
             step(evs[k])
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+        if world > 1:
+            dist.barrier()
+        soak(step, flush, dev, args.soak_s)
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     plan_ms = [e[0].elapsed_time(e[1]) for e in evs]
     scan_ms = [e[1].elapsed_time(e[2]) for e in evs]
@@ -352,6 +367,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=1.0, help="untimed identical steps around the timed ones")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warmup raised to 3 (minimum)")
