@@ -38,7 +38,7 @@ from mla_attention_decode_paged_b200 import workloads as W  # noqa: E402
 DEFAULT_WORKLOAD = "agent_spec"
 METRIC = "MLA decode KV-read GB/s (us/call; % of B200 HBM/tensor roofline)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_simt.cu"]
+KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_sm100.cu"]
 
 
 def log(*a):

@@ -21,7 +21,7 @@ extern "C" mla_status mla_decode_scan(const void* q, const void* kv_pages, int k
         (((uintptr_t)workspace) & 255) || (((uintptr_t)lse) & 3) || (((uintptr_t)block_table) & 3))
         return MLA_ERR_INVALID_ARG;
     if ((int64_t)ws_bytes < make_layout(B, s_q, H, 1).total) return MLA_ERR_WORKSPACE_TOO_SMALL;
-    const int sms = device_sm_count();
+    const int sms = effective_sms();
     if (sms <= 0) return MLA_ERR_CUDA;
 
     DecodeParams p;
@@ -43,6 +43,7 @@ extern "C" mla_status mla_decode_scan(const void* q, const void* kv_pages, int k
     const float ks = kv_dtype == MLA_KV_E4M3 ? kv_scale : 1.f;
     p.score_scale_log2 = scale * ks * kLog2e;
     p.out_scale = ks;
+    if (kv_dtype == MLA_KV_BF16) return launch_decode_sm100(p, (cudaStream_t)stream);
     return launch_decode_simt(p, kv_dtype, (cudaStream_t)stream);
 }
 

@@ -50,7 +50,7 @@ extern "C" mla_status mla_decode_noalloc(const void* q, const void* kv_pages, in
     if (!q || !kv_pages || !block_table || !seq_lens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (B <= 0 || s_q <= 0 || H <= 0) return MLA_ERR_INVALID_ARG;
     if ((int64_t)s_q * H > mla::kMaxRows) return MLA_ERR_UNSUPPORTED;
-    const int sms = mla::device_sm_count();
+    const int sms = mla::effective_sms();
     if (sms <= 0) return MLA_ERR_CUDA;
     const mla::WsLayout L = mla::make_layout(B, s_q, H, mla::num_groups_for(sms, mla::num_row_blocks(s_q, H)));
     if ((size_t)L.total > kScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;

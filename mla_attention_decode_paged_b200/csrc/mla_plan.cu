@@ -11,7 +11,7 @@
 // is found in L2 by the others.
 #include <math.h>
 
-#include "mla_common.cuh"
+#include "mla_decode_params.cuh"
 
 namespace mla {
 
@@ -87,6 +87,15 @@ int device_sm_count() {
     return n;
 }
 
+// SMs the default plan is made for: twice the number of CTA pairs of the scan kernel that
+// the device keeps resident at once (a pair must sit in one GPC, so this can be below the
+// SM count).
+int effective_sms() {
+    int pairs = sm100_pair_slots();
+    if (pairs > 0) return 2 * pairs;
+    return device_sm_count();
+}
+
 bool shape_ok(int B, int s_q, int H) {
     return B > 0 && s_q > 0 && H > 0 && (int64_t)s_q * H <= 65536;
 }
@@ -98,7 +107,7 @@ using namespace mla;
 extern "C" size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms) {
     if (!shape_ok(B, s_q, H) || num_sms < 0) return 0;
     if (num_sms == 0) {
-        num_sms = device_sm_count();
+        num_sms = effective_sms();
         if (num_sms <= 0) return 0;
     }
     WsLayout L = make_layout(B, s_q, H, num_groups_for(num_sms, num_row_blocks(s_q, H)));
@@ -110,7 +119,7 @@ extern "C" mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, i
     if (!seq_lens || !workspace || !shape_ok(B, s_q, H) || num_sms < 0) return MLA_ERR_INVALID_ARG;
     if (((uintptr_t)workspace & 255) != 0) return MLA_ERR_INVALID_ARG;
     if (num_sms == 0) {
-        num_sms = device_sm_count();
+        num_sms = effective_sms();
         if (num_sms <= 0) return MLA_ERR_CUDA;
     }
     if (num_sms < 2) return MLA_ERR_INVALID_ARG;
