@@ -71,7 +71,8 @@ typedef enum { MLA_KV_BF16 = 0, MLA_KV_E4M3 = 1 } mla_kv_dtype;
 /*
  * Bytes of workspace a plan + decode of this shape needs (host, pure).
  * num_sms: SM count the split plan is made for; 0 = the current device's.
- * Returns 0 for an unsupported shape (B, s_q, H <= 0, or s_q * H > 65536).
+ * Returns 0 for an unsupported shape (B, s_q, H <= 0, or s_q * H > 65536) or for a
+ * num_sms that would make more than 1023 groups.
  */
 size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
 
@@ -81,7 +82,7 @@ size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
  * group of SM pairs, cutting requests into splits where a share ends.  The plan is
  * written into `workspace` and is valid for every later mla_decode of the same
  * seq_lens, B, s_q and H (e.g. all layers of one decode step).  num_sms as above; a
- * smaller value gives fewer, longer splits (2 = no splits at all).
+ * smaller value gives fewer, longer splits (1 = no splits at all).
  */
 mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, int H, int num_sms,
                            void* workspace, size_t ws_bytes, void* stream);

@@ -11,62 +11,95 @@
 
 namespace mla {
 
-// grid (B, nqb, 128 / 4), block 128: one warp per folded row, 16 columns per lane.
-__global__ void __launch_bounds__(128) combine_kernel(const void* __restrict__ ws, int B, int s_q, int H,
-                                                      __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+constexpr int kCombineThreads = 512;  // 4 groups of 128 threads; a thread owns one float4 column
+constexpr int kCombineMaxSplits = kMaxGroups + 1;
+
+// grid (B, nqb, 64): one folded row per CTA.  The row's split weights are computed once
+// into shared memory; group j of the CTA accumulates the splits j, j+4, j+8, ... for its
+// float4 column (several independent loads in flight per thread), and the four group
+// sums are added through shared memory.
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __restrict__ ws, int B, int s_q, int H,
+                                                                  __nv_bfloat16* __restrict__ out,
+                                                                  float* __restrict__ lse) {
+    __shared__ float wsh[kCombineMaxSplits];
+    __shared__ float4 part[3][128];
+    __shared__ float red[2];
     const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
     if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
-    const int b = blockIdx.x, qb = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.z * 4 + warp;
+    const int b = blockIdx.x, qb = blockIdx.y, r = blockIdx.z;
     const int M = s_q * H;
     const int row = qb * kRowsPerBlock + r;
     if (row >= M) return;
     const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
-    const int s0 = req_seg[b], s1 = req_seg[b + 1];
-    if (s1 - s0 <= 1) return;  // written directly by the decode kernel
+    const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
+    if (ns <= 1) return;  // written directly by the decode kernel
     const int nqb = h->nqb;
     const float* plse = ws_ptr<float>(ws, h->off_plse);
     const float* po = ws_ptr<float>(ws, h->off_po);
+    const int64_t stride = (int64_t)nqb * kRowsPerBlock;  // rows between consecutive segments
+    const int64_t prow0 = ((int64_t)s0 * nqb + qb) * kRowsPerBlock + r;
+    const int tid = threadIdx.x, grp = tid >> 7, c4 = tid & 127;
 
-    float mx = -INFINITY;
-    for (int s = s0; s < s1; ++s) mx = fmaxf(mx, plse[((int64_t)s * nqb + qb) * kRowsPerBlock + r]);
-    float sum = 0.f;
-    if (mx != -INFINITY)
-        for (int s = s0; s < s1; ++s) sum += fast_exp2(plse[((int64_t)s * nqb + qb) * kRowsPerBlock + r] - mx);
-    const float L = mx + __log2f(sum);
-
-    float4 acc[4];
+    // L = log2 sum_j 2^lse2_j and the weights 2^(lse2_j - L), by warp 0
+    if (tid < 32) {
+        float mx = -INFINITY;
+        for (int j = tid; j < ns; j += 32) mx = fmaxf(mx, plse[prow0 + j * stride]);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = s0; s < s1; ++s) {
-        const int64_t prow = ((int64_t)s * nqb + qb) * kRowsPerBlock + r;
-        const float l2 = plse[prow];
-        if (l2 == -INFINITY) continue;
-        const float w = fast_exp2(l2 - L);
-        const float4* src = reinterpret_cast<const float4*>(po + prow * kDv);
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+        if (mx != -INFINITY)
+            for (int j = tid; j < ns; j += 32) sum += fast_exp2(plse[prow0 + j * stride] - mx);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float4 v = src[lane + 32 * k];
-            acc[k].x += w * v.x; acc[k].y += w * v.y; acc[k].z += w * v.z; acc[k].w += w * v.w;
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float L = mx + __log2f(sum);
+        for (int j = tid; j < ns && j < kCombineMaxSplits; j += 32) {
+            const float l2 = plse[prow0 + j * stride];
+            wsh[j] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - L);  // an empty split drops out
+        }
+        if (tid == 0) {
+            red[0] = L;
+            red[1] = mx;
         }
     }
-    __nv_bfloat16* dst = out + ((int64_t)b * M + row) * kDv;
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int j = grp;
+    for (; j + 12 < ns; j += 16) {
+        float4 v[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[k].x, acc[k].y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[k].z, acc[k].w);
+        for (int u = 0; u < 4; ++u) v[u] = reinterpret_cast<const float4*>(po + (prow0 + (int64_t)(j + 4 * u) * stride) * kDv)[c4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float w = wsh[j + 4 * u];
+            acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+        }
+    }
+    for (; j < ns; j += 4) {
+        const float4 v = reinterpret_cast<const float4*>(po + (prow0 + (int64_t)j * stride) * kDv)[c4];
+        const float w = wsh[j];
+        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+    }
+    if (grp > 0) part[grp - 1][c4] = acc;
+    __syncthreads();
+    if (grp == 0) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const float4 v = part[k][c4];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
         uint2 pk;
         pk.x = *reinterpret_cast<uint32_t*>(&lo);
         pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(dst + 4 * (lane + 32 * k)) = pk;
+        *reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDv + 4 * c4) = pk;
+        if (c4 == 0) lse[(int64_t)b * M + row] = (red[1] == -INFINITY) ? -INFINITY : red[0] * kLn2;
     }
-    if (lane == 0) lse[(int64_t)b * M + row] = (mx == -INFINITY) ? -INFINITY : L * kLn2;
 }
 
 mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream) {
-    dim3 grid(B, num_row_blocks(s_q, H), kRowsPerBlock / 4);
-    combine_kernel<<<grid, 128, 0, stream>>>(ws, B, s_q, H, reinterpret_cast<__nv_bfloat16*>(out), lse);
+    dim3 grid(B, num_row_blocks(s_q, H), kRowsPerBlock);
+    combine_kernel<<<grid, kCombineThreads, 0, stream>>>(ws, B, s_q, H, reinterpret_cast<__nv_bfloat16*>(out), lse);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

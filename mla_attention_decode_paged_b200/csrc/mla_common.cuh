@@ -15,8 +15,9 @@ namespace mla {
 constexpr int kDqk = MLA_HEAD_DIM_QK;  // 512 latent + 64 rope
 constexpr int kDv = MLA_HEAD_DIM_V;
 constexpr int kPage = MLA_PAGE_SIZE;
-constexpr int kRowsPerBlock = 128;     // folded query rows per row block (one MMA M tile)
+constexpr int kRowsPerBlock = 64;      // folded query rows per row block (one CTA, MMA M = 64)
 constexpr int kMaxRows = 256;          // s_q * H supported per request
+constexpr int kMaxGroups = 1023;       // plan groups (a request has at most groups + 1 splits)
 constexpr int32_t kPlanMagic = 0x4d4c4131;  // "MLA1"
 
 // Device-side error codes (mirror mla_status values).
@@ -38,7 +39,7 @@ struct __align__(16) PlanHeader {
     int32_t magic;
     int32_t B, s_q, H;
     int32_t nqb;          // row blocks per request: ceil(s_q*H / 128)
-    int32_t num_groups;   // groups of SM pairs; all pairs of a group scan the same pages
+    int32_t num_groups;   // groups of CTAs; all CTAs of a group scan the same pages
     int32_t num_segments;
     int32_t max_segments;
     int32_t total_tiles;
@@ -46,8 +47,8 @@ struct __align__(16) PlanHeader {
     int64_t off_group_begin;  // int32 [num_groups + 1]
     int64_t off_req_seg;      // int32 [B + 1]
     int64_t off_segs;         // Segment [max_segments]
-    int64_t off_plse;         // float [max_segments][nqb][128]   (log2 domain)
-    int64_t off_po;           // float [max_segments][nqb][128][512]
+    int64_t off_plse;         // float [max_segments][nqb][64]   (log2 domain)
+    int64_t off_po;           // float [max_segments][nqb][64][512]
     int64_t total_bytes;
 };
 
@@ -62,11 +63,11 @@ __host__ __device__ inline int num_row_blocks(int s_q, int H) {
     return (s_q * H + kRowsPerBlock - 1) / kRowsPerBlock;
 }
 
-// Groups of SM pairs for a device with num_sms SMs: every group holds nqb pairs (one
-// per row block) so that the pairs of a group read the same pages at the same time.
+// Groups of CTAs for a device with num_sms SMs (one scan CTA per SM): every group holds
+// nqb CTAs (one per row block) so that the CTAs of a group read the same pages at the
+// same time and share them through L2.
 __host__ __device__ inline int num_groups_for(int num_sms, int nqb) {
-    int pairs = num_sms / 2;
-    int g = pairs / nqb;
+    int g = num_sms / nqb;
     return g < 1 ? 1 : g;
 }
 

@@ -43,8 +43,7 @@ extern "C" mla_status mla_decode_scan(const void* q, const void* kv_pages, int k
     const float ks = kv_dtype == MLA_KV_E4M3 ? kv_scale : 1.f;
     p.score_scale_log2 = scale * ks * kLog2e;
     p.out_scale = ks;
-    if (kv_dtype == MLA_KV_BF16) return launch_decode_sm100(p, (cudaStream_t)stream);
-    return launch_decode_simt(p, kv_dtype, (cudaStream_t)stream);
+    return launch_decode_sm100(p, kv_dtype, (cudaStream_t)stream);
 }
 
 extern "C" mla_status mla_decode(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,

@@ -24,10 +24,10 @@ struct DecodeParams {
 };
 
 mla_status launch_decode_simt(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
-mla_status launch_decode_sm100(const DecodeParams& p, cudaStream_t stream);
-// Pairs (2-CTA clusters) of the tensor-core scan kernel that the current device runs at
-// once; 2 x this is the SM count the split plan is made for by default.
-int sm100_pair_slots();
+mla_status launch_decode_sm100(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
+// CTAs of the tensor-core scan kernel that the current device runs at once (one per
+// SM); the split plan is made for this many by default.
+int sm100_cta_slots();
 int effective_sms();
 mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream);
 int device_sm_count();

@@ -1,32 +1,31 @@
 // mla_decode_sm100.cu -- the split scan of paged absorbed-MLA decode on Blackwell
 // tensor cores (tcgen05 + TMEM + TMA), sm_100a.
 //
-// Work unit.  A cluster of two CTAs (a "pair", one CTA per SM) owns one block of 128
-// folded query rows (row m = i * H + h, the query-sequence axis folded into the head
-// axis so that the MMA M tile is full: "TokenSpeed" launch digest, MLA kernel
-// paragraphs) of one split of one request, and walks the split's 64-token pages.
+// Work unit.  One CTA (one per SM) owns a block of 64 folded query rows (row
+// m = i * H + h: the query-sequence axis folded into the head axis, "TokenSpeed" launch
+// digest, MLA kernel paragraphs) of one split of one request, and walks the split's
+// 64-token pages.  There is no cross-CTA traffic: the CTAs of a plan group read the
+// same pages at the same time and share them through L2.
 //
-// Column split.  The 576-wide score contraction and the 512-wide output are divided
-// between the two CTAs: CTA c holds latent columns [256c, 256c+256) and RoPE columns
-// [512+32c, 512+32c+32) of q and of every cached row (288 columns, 72 KB of q), and it
-// accumulates out[:, 256c:256c+256] in tensor memory.  Each CTA computes the partial
-// score S_c = q[:, cols_c] . KV[:, cols_c]^T of a page, the two CTAs swap partials
-// through distributed shared memory, and both add them in the same order, so both hold
-// bit-identical scores and take identical softmax decisions.  Every score and output
-// FLOP is done once, and each CTA loads only its own 288 columns of each page.
-//
-// Per CTA and page (64 tokens):
-//   TMA (producer warp): 4 latent boxes [64 tok x 64 col] (128-byte swizzle) and one RoPE
-//       box [64 x 32] (64-byte swizzle) of the physical page block_table[b][p].
-//   MMA (one thread): S = Q_c . K_c^T, M=128 N=64, 18 K-steps of 16, into TMEM;
-//       later O += P . V_c, M=128 N=256, 4 K-steps, with P read from TMEM and V the same
-//       shared-memory page viewed MN-major.
-//   softmax (4 warps, one thread per row): partial S from TMEM, exchange, base-2 online
-//       softmax with the causal draft mask, P in bf16 back into TMEM over its S columns.
-//       The running maximum is only raised (and O rescaled) when a new score exceeds it
-//       by more than 8 in base 2, so P <= 256 and rescales are rare.
-//   epilogue: O / l -> bf16 out (request held whole by this split) or fp32 partial + lse2
-//       (split request; merged by the combine kernel).
+// Tensor memory (128 lanes x 512 columns) with 64-row MMAs, whose rows occupy 16 lanes
+// of each 32-lane subpartition:
+//   lanes at offset 0  : O, the 64 x 512 fp32 output accumulator (all 512 columns)
+//   lanes at offset 16 : q (64 x 576 bf16, 288 columns, loaded once per split) and two
+//                        64-column score buffers.
+// Per page:
+//   TMA (producer warp): the page's 64 rows x 576 columns as nine 64-column boxes with
+//       128-byte swizzle (one 72 KB stage; three stages).  An e4m3 page lands as nine
+//       unswizzled 64 x 64-byte boxes in the upper half of each bf16 slot, and four more
+//       warps widen it to bf16 in place (exact); kv_scale is folded into the score and
+//       output scales.
+//   MMA (one thread): S = q . K^T with q read from TMEM (M=64 N=64, 36 K-steps), then
+//       O += P . V with P (bf16) and V (the same page, read MN-major) from shared memory
+//       (M=64 N=256, twice, 4 K-steps each).
+//   softmax (4 warps, 16 rows each, two threads per row with 32 scores each): base-2
+//       online softmax with the causal draft mask; the running max is only raised (and
+//       O rescaled) when a score exceeds it by more than 8, so P <= 256.
+//   epilogue: O / l -> bf16 out (a request the split holds whole) or an fp32 partial and
+//       its base-2 lse (split request; merged by the combine kernel).
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
@@ -39,53 +38,54 @@
 namespace mla {
 namespace {
 
-constexpr int kRows = 128;       // folded query rows per pair (MMA M)
-constexpr int kTok = 64;         // tokens per page / tile (S MMA N)
-constexpr int kStages = 3;       // cache pages in flight per CTA
-constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue
+constexpr int kRows = kRowsPerBlock;  // 64 folded rows per CTA (MMA M)
+constexpr int kTok = 64;              // tokens per page (S MMA N)
+constexpr int kStages = 3;
+// warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue, and for an e4m3 cache warps 6-9
+// widen each landed page to bf16 in place
+constexpr int kThreadsBf16 = 192;
+constexpr int kThreadsE4m3 = 320;
+template <int KV>
+constexpr int threads_for() { return KV == MLA_KV_E4M3 ? kThreadsE4m3 : kThreadsBf16; }
+static_assert(kRows == 64, "the TMEM layout below is the 64-row MMA layout");
 
-constexpr uint32_t kQLatChunk = kRows * 128;                  // 128 rows x 64 bf16
-constexpr uint32_t kQRope = kRows * 64;                       // 128 rows x 32 bf16
-constexpr uint32_t kQBytes = 4 * kQLatChunk + kQRope;         // 73,728
-constexpr uint32_t kKvLatChunk = kTok * 128;                  // 64 tokens x 64 bf16
-constexpr uint32_t kKvRope = kTok * 64;                       // 64 tokens x 32 bf16
-constexpr uint32_t kStageBytes = 4 * kKvLatChunk + kKvRope;   // 36,864
-constexpr uint32_t kXchgBytes = kRows * kTok * 4;             // fp32 partial scores
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKv = kOffQ + kQBytes;
-constexpr uint32_t kOffXchg = kOffKv + kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffXchg + kXchgBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;         // barriers + alignment slack
+constexpr uint32_t kChunk = kTok * 128;              // 64 tokens x 64 columns bf16, 128B-swizzled
+constexpr uint32_t kStageBytes = 9 * kChunk;         // 8 latent chunks + 1 rope chunk: 72 KB
+constexpr uint32_t kRawChunk = kTok * 64;            // e4m3: 64 tokens x 64 columns, in the upper half
+constexpr uint32_t kRawStageBytes = 9 * kRawChunk;   //        of each bf16 chunk slot
+constexpr uint32_t kPBytes = kRows * kTok * 2;       // P: 64 rows x 64 tokens bf16
+constexpr uint32_t kOffKv = 0;
+constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffP + kPBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 
-// mbarrier slots (8 bytes each)
 enum : int {
-    B_Q_FULL = 0, B_Q_EMPTY, B_KV_FULL0, B_KV_EMPTY0 = B_KV_FULL0 + kStages, B_S_FULL0 = B_KV_EMPTY0 + kStages,
-    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_O_EMPTY = B_PV_DONE0 + 2, B_XFULL, B_XEMPTY,
-    B_SMSYNC, B_DRAIN, B_COUNT
+    B_KV_FULL0 = 0, B_KV_EMPTY0 = B_KV_FULL0 + kStages, B_Q_FULL = B_KV_EMPTY0 + kStages, B_S_FULL0,
+    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_DRAIN = B_PV_DONE0 + 2, B_RAW0,
+    B_CONV = B_RAW0 + kStages, B_COUNT
 };
 constexpr uint32_t kOffTmemHolder = kOffBar + 8 * B_COUNT;
 constexpr uint32_t kOffAbort = kOffTmemHolder + 4;
 static_assert(kOffAbort + 4 <= kOffBar + 256, "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;     // 256 columns: out[:, 256c : 256c+256] accumulator
-constexpr uint32_t kTmemS = 256;   // 2 x 64 columns: scores, then P (bf16 pairs) in place
-constexpr float kRescaleThreshold = 8.0f;  // base-2 headroom before the running max is raised
+constexpr uint32_t kLaneHi = 16u << 16;  // second half-subpartition set (q and scores)
+constexpr uint32_t kColQ = 0;            // q: 288 columns (bf16 pairs)
+constexpr uint32_t kColS = 288;          // scores: 2 x 64 columns
+constexpr float kRescaleThreshold = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRows, kTok, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kRows, 256, 0, 1);
 
 struct __align__(64) Sm100Args {
-    CUtensorMap tm_q_lat;    // q viewed [B*M rows, 576], box 64 cols x 128 rows, 128B swizzle
-    CUtensorMap tm_q_rope;   // box 32 x 128, 64B swizzle
-    CUtensorMap tm_kv_lat;   // cache viewed [P*64 rows, 576], box 64 x 64, 128B swizzle
-    CUtensorMap tm_kv_rope;  // box 32 x 64, 64B swizzle
+    CUtensorMap tm_kv;  // cache viewed [P*64 rows, 576 cols]: bf16 box 64 x 64 with 128B swizzle, or
+                        // e4m3 box 64 x 64 bytes without swizzle
     DecodeParams p;
 };
 
 struct Ctx {
-    uint32_t bar0;            // shared address of barrier 0
+    uint32_t bar0;
     volatile int* abort;
     PlanHeader* h;
     __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
@@ -93,15 +93,14 @@ struct Ctx {
 
 // Bounded wait: gives up after kWaitLimitNs (sets the timeout status and the CTA abort
 // flag), or at once once the CTA is aborting.
-__device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool cluster_scope) {
+__device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
     if (*c.abort) return false;
     uint64_t t0 = 0;
     for (uint32_t n = 1;; ++n) {
-        bool ok = cluster_scope ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
-        if (ok) return true;
+        if (ptx::mbar_try_wait(bar, parity)) return true;
         if ((n & 255) == 0) {
             if (*c.abort) return false;
-            uint64_t now = ptx::globaltimer_ns();
+            const uint64_t now = ptx::globaltimer_ns();
             if (t0 == 0) {
                 t0 = now;
             } else if (now - t0 > kWaitLimitNs) {
@@ -115,7 +114,7 @@ __device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parit
 
 // Wait that ignores the abort flag, used only on the way out for work already in flight.
 __device__ void drain_wait(uint32_t bar, uint32_t parity) {
-    uint64_t t0 = ptx::globaltimer_ns();
+    const uint64_t t0 = ptx::globaltimer_ns();
     while (!ptx::mbar_try_wait(bar, parity)) {
         if (ptx::globaltimer_ns() - t0 > 200000000ull) return;
     }
@@ -130,8 +129,36 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    decode_sm100_kernel(const __grid_constant__ Sm100Args args) {
+// Twelve score K-steps starting at K0 (of 36): q from TMEM, the page from shared memory.
+// K0 is a template constant so that every descriptor offset is an immediate.
+template <int K0>
+__device__ __forceinline__ void issue_s_chunk(uint32_t d, uint32_t a0, uint64_t b0) {
+#pragma unroll
+    for (int k = 0; k < 12; ++k) {
+        constexpr int kChunkUnits = kChunk >> 4;
+        const int ks = K0 + k;
+        ptx::mma_ts(d, a0 + 8u * ks, b0 + (uint64_t)((ks >> 2) * kChunkUnits + (ks & 3) * 2), kIdescS,
+                    ks ? 1u : 0u);
+    }
+}
+
+// e4m3 -> bf16 for 32 consecutive bytes (exact: every e4m3 value is a bf16 value)
+__device__ __forceinline__ void widen_e4m3x32(const uint4 (&in)[2], uint32_t (&out)[16]) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        const uint32_t word = (w < 4) ? (&in[0].x)[w] : (&in[1].x)[w - 4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float2 f = e4m3x2_to_float2((uint16_t)(word >> (16 * hh)));
+            __nv_bfloat162 v = __floats2bfloat162_rn(f.x, f.y);
+            out[2 * w + hh] = *reinterpret_cast<uint32_t*>(&v);
+        }
+    }
+}
+
+template <int KV>
+__global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(const __grid_constant__ Sm100Args args) {
+    constexpr bool kE4m3 = KV == MLA_KV_E4M3;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
@@ -142,48 +169,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (h->magic != kPlanMagic || h->B != p.B || h->s_q != p.s_q || h->H != p.H ||
         h->num_groups > p.groups_launched) {
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(h, kStatusPlanMismatch, 0);
-        return;  // both CTAs of every pair see the same header
+        return;
     }
     const int nqb = h->nqb;
-    const int pair = blockIdx.x >> 1;
-    const int g = pair / nqb, qb = pair % nqb;
+    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
     if (g >= h->num_groups) return;
-    const uint32_t crank = ptx::cluster_ctarank();
-    const uint32_t peer = crank ^ 1u;
 
     Ctx c;
     c.bar0 = sbase + kOffBar;
     c.abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
     c.h = h;
-
     if (threadIdx.x == 0) {
         *c.abort = 0;
-        ptx::mbar_init(c.bar(B_Q_FULL), 1);
-        ptx::mbar_init(c.bar(B_Q_EMPTY), 1);
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(c.bar(B_KV_FULL0 + s), 1);
+            // bf16: the TMA completes the stage; e4m3: the 128 converter threads do
+            ptx::mbar_init(c.bar(B_KV_FULL0 + s), kE4m3 ? 128 : 1);
             ptx::mbar_init(c.bar(B_KV_EMPTY0 + s), 1);
+            ptx::mbar_init(c.bar(B_RAW0 + s), 1);
         }
+        ptx::mbar_init(c.bar(B_CONV), 128);
+        ptx::mbar_init(c.bar(B_Q_FULL), 128);
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(c.bar(B_S_FULL0 + s), 1);
             ptx::mbar_init(c.bar(B_P_READY0 + s), 128);
             ptx::mbar_init(c.bar(B_PV_DONE0 + s), 1);
         }
-        ptx::mbar_init(c.bar(B_O_EMPTY), 128);
-        ptx::mbar_init(c.bar(B_XFULL), 1);
-        ptx::mbar_init(c.bar(B_XEMPTY), 1);
-        ptx::mbar_init(c.bar(B_SMSYNC), 128);
         ptx::mbar_init(c.bar(B_DRAIN), 1);
         ptx::fence_mbar_init_cluster();
-        // arm the first exchange phase: the peer's partial scores complete it
-        ptx::mbar_arrive_expect_tx(c.bar(B_XFULL), kXchgBytes);
     }
-    if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&args.tm_q_lat);
-        ptx::prefetch_tmap(&args.tm_q_rope);
-        ptx::prefetch_tmap(&args.tm_kv_lat);
-        ptx::prefetch_tmap(&args.tm_kv_rope);
-    }
+    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
     if (warp == 1) {
         ptx::tmem_alloc(sbase + kOffTmemHolder, kTmemCols);
         ptx::tmem_relinquish();
@@ -191,7 +205,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    ptx::cluster_sync();  // the peer's barriers exist before any remote arrive or st.async
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemHolder);
 
     const int32_t* group_begin = ws_ptr<int32_t>(p.ws, h->off_group_begin);
@@ -201,45 +214,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int it = 0, nseg = 0;
+            int it = 0;
             for (int si = seg_lo; si < seg_hi && !*c.abort; ++si) {
                 const Segment S = segs[si];
                 const int T = p.seq_lens[S.b];
                 if (!request_ok(p, T)) continue;
-                if (nseg > 0 && !wait_bar(c, c.bar(B_Q_EMPTY), (nseg - 1) & 1, false)) break;
-                const int qy = S.b * p.M + qb * kRows;
-                ptx::mbar_arrive_expect_tx(c.bar(B_Q_FULL), kQBytes);
-                for (int j = 0; j < 4; ++j)
-                    ptx::tma_load_2d(sbase + kOffQ + j * kQLatChunk, &args.tm_q_lat, c.bar(B_Q_FULL),
-                                     256 * (int)crank + 64 * j, qy);
-                ptx::tma_load_2d(sbase + kOffQ + 4 * kQLatChunk, &args.tm_q_rope, c.bar(B_Q_FULL),
-                                 512 + 32 * (int)crank, qy);
+                bool ok = true;
                 for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
                     const int st = it % kStages;
-                    if (it >= kStages && !wait_bar(c, c.bar(B_KV_EMPTY0 + st), ((it / kStages) - 1) & 1, false))
+                    if (it >= kStages && !wait_bar(c, c.bar(B_KV_EMPTY0 + st), ((it / kStages) - 1) & 1)) {
+                        ok = false;
                         break;
+                    }
                     const int32_t page = p.block_table[(int64_t)S.b * p.max_pages + t];
-                    // an invalid page id becomes a fully out-of-range box (zero fill); the
-                    // softmax warps see the same id and poison the rows
+                    // an invalid page id becomes a box entirely out of range (zero fill); the
+                    // softmax warps see the same id and poison the request's rows
                     const int ky = (page >= 0 && page < p.num_pages) ? page * kPage : -kPage;
                     const uint32_t dst = sbase + kOffKv + st * kStageBytes;
-                    ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
-                    for (int j = 0; j < 4; ++j)
-                        ptx::tma_load_2d(dst + j * kKvLatChunk, &args.tm_kv_lat, c.bar(B_KV_FULL0 + st),
-                                         256 * (int)crank + 64 * j, ky);
-                    ptx::tma_load_2d(dst + 4 * kKvLatChunk, &args.tm_kv_rope, c.bar(B_KV_FULL0 + st),
-                                     512 + 32 * (int)crank, ky);
+                    if (kE4m3) {
+                        ptx::mbar_arrive_expect_tx(c.bar(B_RAW0 + st), kRawStageBytes);
+#pragma unroll
+                        for (int j = 0; j < 9; ++j)
+                            ptx::tma_load_2d(dst + j * kChunk + kRawChunk, &args.tm_kv, c.bar(B_RAW0 + st), 64 * j, ky);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
+#pragma unroll
+                        for (int j = 0; j < 9; ++j)
+                            ptx::tma_load_2d(dst + j * kChunk, &args.tm_kv, c.bar(B_KV_FULL0 + st), 64 * j, ky);
+                    }
                 }
-                ++nseg;
+                if (!ok) break;
             }
             if (*c.abort) {
-                // let loads already issued land before the CTA goes away
                 for (int k = (it > kStages ? it - kStages : 0); k < it; ++k)
-                    drain_wait(c.bar(B_KV_FULL0 + k % kStages), (k / kStages) & 1);
+                    drain_wait(c.bar((kE4m3 ? B_RAW0 : B_KV_FULL0) + k % kStages), (k / kStages) & 1);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // An event loop: the score MMAs of the next page and the PV MMAs of the oldest
+        // page whose P is ready are issued in whichever order their inputs arrive, so a
+        // stage is released as soon as its PV completes instead of waiting behind the
+        // next page's load.  The tensor core runs them in issue order.  Barriers are
+        // polled with test_wait, which never suspends the thread.
         if (lane == 0) {
             int it = 0, nseg = 0;
             bool ok = true;
@@ -247,77 +264,141 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const Segment S = segs[si];
                 const int T = p.seq_lens[S.b];
                 if (!request_ok(p, T)) continue;
-                if (!wait_bar(c, c.bar(B_Q_FULL), nseg & 1, false)) break;
+                if (!wait_bar(c, c.bar(B_Q_FULL), nseg & 1)) break;
                 ptx::tc_fence_after();
                 const int n = S.tile_end - S.tile_begin;
-                auto issue_pv = [&](int itp, bool first) -> bool {
-                    if (first && nseg > 0 && !wait_bar(c, c.bar(B_O_EMPTY), (nseg - 1) & 1, false)) return false;
-                    if (!wait_bar(c, c.bar(B_P_READY0 + (itp & 1)), (itp >> 1) & 1, false)) return false;
-                    ptx::tc_fence_after();
-                    const uint32_t vbase = sbase + kOffKv + (itp % kStages) * kStageBytes;
-                    const uint32_t a_tmem = tmem + kTmemS + 64u * (itp & 1);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        // V = the page's latent columns, MN-major: 64-column blocks 8 KB apart
-                        // (leading offset), 8-token groups 1 KB apart (stride offset)
-                        const uint64_t bdesc = ptx::smem_desc(vbase + ks * 2048, kKvLatChunk, 1024, ptx::kSwizzle128);
-                        ptx::mma_ts(tmem + kTmemO, a_tmem + 8 * ks, bdesc, kIdescPV, (first && ks == 0) ? 0u : 1u);
-                    }
-                    ptx::mma_commit(c.bar(B_PV_DONE0 + (itp & 1)));
-                    ptx::mma_commit(c.bar(B_KV_EMPTY0 + (itp % kStages)));
-                    return true;
-                };
-                for (int jj = 0; jj < n && ok; ++jj, ++it) {
-                    const int st = it % kStages;
-                    if (!wait_bar(c, c.bar(B_KV_FULL0 + st), (it / kStages) & 1, false)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t kbase = sbase + kOffKv + st * kStageBytes;
-                    const uint32_t d = tmem + kTmemS + 64u * (it & 1);
-#pragma unroll
-                    for (int kc = 0; kc < 4; ++kc) {
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint64_t a = ptx::smem_desc(sbase + kOffQ + kc * kQLatChunk + ks * 32, 16, 1024,
-                                                              ptx::kSwizzle128);
-                            const uint64_t b = ptx::smem_desc(kbase + kc * kKvLatChunk + ks * 32, 16, 1024,
-                                                              ptx::kSwizzle128);
-                            ptx::mma_ss(d, a, b, kIdescS, (kc | ks) ? 1u : 0u);
+                int ns = 0, npv = 0;  // pages of this split with S issued / PV issued
+                uint64_t t0 = 0;
+                uint32_t spins = 0;
+                while (npv < n) {
+                    bool progressed = false;
+                    // S(ns) reuses the score buffer of page ns-2, whose PV must be issued first
+                    if (ns < n && ns <= npv + 1) {
+                        const int its = it + ns, st = its % kStages;
+                        if (ptx::mbar_test_wait(c.bar(B_KV_FULL0 + st), (its / kStages) & 1)) {
+                            ptx::tc_fence_after();
+                            // descriptors are built once and advanced by constant 16-byte offsets:
+                            // the fully unrolled issue loop is a handful of integer adds per MMA
+                            const uint64_t b0 = ptx::smem_desc(sbase + kOffKv + st * kStageBytes, 16, 1024,
+                                                               ptx::kSwizzle128);
+                            const uint32_t d = tmem + kLaneHi + kColS + 64u * (its & 1);
+                            const uint32_t a0 = tmem + kLaneHi + kColQ;
+                            issue_s_chunk<0>(d, a0, b0);
+                            issue_s_chunk<12>(d, a0, b0);
+                            issue_s_chunk<24>(d, a0, b0);
+                            ptx::mma_commit(c.bar(B_S_FULL0 + (its & 1)));
+                            ++ns;
+                            progressed = true;
                         }
                     }
+                    if (npv < ns) {
+                        const int itp = it + npv;
+                        if (ptx::mbar_test_wait(c.bar(B_P_READY0 + (itp & 1)), (itp >> 1) & 1)) {
+                            ptx::tc_fence_after();
+                            const bool first = npv == 0;
+                            // A = P (K-major); B = V, MN-major: 64-column blocks 8 KB apart (leading
+                            // offset), 8-token groups 1 KB apart (stride offset)
+                            const uint64_t a0 = ptx::smem_desc(sbase + kOffP, 16, 1024, ptx::kSwizzle128);
+                            const uint64_t v0 = ptx::smem_desc(sbase + kOffKv + (itp % kStages) * kStageBytes, kChunk,
+                                                               1024, ptx::kSwizzle128);
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        const uint64_t a = ptx::smem_desc(sbase + kOffQ + 4 * kQLatChunk + ks * 32, 16, 512,
-                                                          ptx::kSwizzle64);
-                        const uint64_t b = ptx::smem_desc(kbase + 4 * kKvLatChunk + ks * 32, 16, 512, ptx::kSwizzle64);
-                        ptx::mma_ss(d, a, b, kIdescS, 1u);
+                            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    ptx::mma_ss(tmem + 256u * half, a0 + (uint64_t)(ks * 2),
+                                                v0 + (uint64_t)(half * 4 * (kChunk >> 4) + ks * (2048 >> 4)), kIdescPV,
+                                                (first && ks == 0) ? 0u : 1u);
+                            }
+                            ptx::mma_commit(c.bar(B_PV_DONE0 + (itp & 1)));
+                            ptx::mma_commit(c.bar(B_KV_EMPTY0 + (itp % kStages)));
+                            ++npv;
+                            progressed = true;
+                        }
                     }
-                    ptx::mma_commit(c.bar(B_S_FULL0 + (it & 1)));
-                    if (jj > 0 && !issue_pv(it - 1, jj == 1)) { ok = false; break; }
+                    if (progressed) {
+                        t0 = 0;
+                        spins = 0;
+                    } else if ((++spins & 255) == 0) {
+                        // same bound as every other wait in this kernel
+                        if (*c.abort) { ok = false; break; }
+                        const uint64_t now = ptx::globaltimer_ns();
+                        if (t0 == 0) {
+                            t0 = now;
+                        } else if (now - t0 > kWaitLimitNs) {
+                            *c.abort = 1;
+                            set_status(h, kStatusTimeout, (int)blockIdx.x);
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
-                if (!ok) break;
-                if (!issue_pv(it - 1, n == 1)) break;
-                ptx::mma_commit(c.bar(B_Q_EMPTY));
+                it += n;
                 ++nseg;
             }
             ptx::mma_commit(c.bar(B_DRAIN));
             drain_wait(c.bar(B_DRAIN), 0);
         }
+    } else if (kE4m3 && warp >= 6) {
+        // ------------------------------------------------------------ e4m3 -> bf16 (warps 6-9)
+        // Every thread takes one half-row (32 bytes) of each of the nine chunks: all reads
+        // first, a bounded barrier among the converters, then the writes, because each bf16
+        // chunk overwrites its own e4m3 bytes in the upper half of its slot.
+        const int ct = threadIdx.x - 192;  // 0..127
+        const int r = ct >> 1, hf = ct & 1;
+        int it = 0;
+        bool alive = true;
+        for (int si = seg_lo; si < seg_hi && alive; ++si) {
+            const Segment S = segs[si];
+            const int T = p.seq_lens[S.b];
+            if (!request_ok(p, T)) continue;
+            for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
+                const int st = it % kStages;
+                alive = wait_bar(c, c.bar(B_RAW0 + st), (it / kStages) & 1);
+                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
+                uint8_t* stage = smem + kOffKv + st * kStageBytes;
+                uint4 raw[9][2];
+#pragma unroll
+                for (int j = 0; j < 9; ++j) {
+                    const uint4* src = reinterpret_cast<const uint4*>(stage + j * kChunk + kRawChunk + r * 64 + hf * 32);
+                    raw[j][0] = src[0];
+                    raw[j][1] = src[1];
+                }
+                ptx::mbar_arrive(c.bar(B_CONV));
+                alive = wait_bar(c, c.bar(B_CONV), it & 1);
+                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
+#pragma unroll
+                for (int j = 0; j < 9; ++j) {
+                    uint32_t o[16];
+                    widen_e4m3x32(raw[j], o);
+                    uint8_t* rowp = stage + j * kChunk + r * 128;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int piece = 4 * hf + w;  // 16-byte piece of the 128-byte row, swizzled
+                        *reinterpret_cast<uint4*>(rowp + ((piece ^ (r & 7)) << 4)) =
+                            make_uint4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(c.bar(B_KV_FULL0 + st));
+            }
+        }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
-        const int row = quad * 32 + lane;          // folded row within the block
-        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        const int tid = threadIdx.x - 64;          // 0..127
-        const uint32_t xchg_local = sbase + kOffXchg;
-        const uint32_t xchg_remote = ptx::mapa(xchg_local, peer);
-        const uint32_t xfull_remote = ptx::mapa(c.bar(B_XFULL), peer);
-        const uint32_t xempty_remote = ptx::mapa(c.bar(B_XEMPTY), peer);
-        const float* xchg_f = reinterpret_cast<const float*>(smem + kOffXchg);
+        const int quad = warp & 3;             // TMEM lane quadrant this warp may access
+        const int r16 = lane & 15;
+        const int half = lane >> 4;            // score columns [32 half, +32), output columns [32 half + 64 q, +32)
+        const int row = quad * 16 + r16;       // folded row within the block
+        const uint32_t t_hi = tmem + ((uint32_t)(quad * 32) << 16) + kLaneHi;  // q and scores
+        const uint32_t t_lo = tmem + ((uint32_t)(quad * 32) << 16);            // O
+        const int tid = threadIdx.x - 64;      // 0..127
         const int m_glob = qb * kRows + row;
         const bool row_valid = m_glob < p.M;
+        const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(p.q);
         float* plse = ws_ptr<float>(p.ws, h->off_plse);
         float* po = ws_ptr<float>(p.ws, h->off_po);
-        int it = 0, nseg = 0;
+        uint8_t* pbuf = smem + kOffP;
+        int it = 0;
+        bool alive = true;
 
         for (int si = seg_lo; si < seg_hi; ++si) {
             const Segment S = segs[si];
@@ -329,73 +410,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (row_valid) {
                     const float nanv = __int_as_float(0x7fc00000);
                     if (!S.split) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * kDv + 256 * crank;
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * kDv + 256 * half;
                         for (int k = 0; k < 256; ++k) dst[k] = __float2bfloat16_rn(nanv);
-                        if (crank == 0) p.lse[orow] = nanv;
+                        if (half == 0) p.lse[orow] = nanv;
                     } else {
-                        float* dst = po + prow * kDv + 256 * crank;
+                        float* dst = po + prow * kDv + 256 * half;
                         for (int k = 0; k < 256; ++k) dst[k] = nanv;
-                        if (crank == 0) plse[prow] = nanv;
+                        if (half == 0) plse[prow] = nanv;
                     }
                 }
                 continue;
             }
             if (*c.abort) break;
+            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + m_glob) * kDqk);
+#pragma unroll 1
+                for (int k = 0; k < 9; ++k) {
+                    uint32_t v[16];
+                    const int d0 = 64 * k + 32 * half;  // first of this thread's 32 dims
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint4 x = row_valid ? src[d0 / 8 + w] : make_uint4(0, 0, 0, 0);
+                        v[4 * w] = x.x;
+                        v[4 * w + 1] = x.y;
+                        v[4 * w + 2] = x.z;
+                        v[4 * w + 3] = x.w;
+                    }
+                    ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * k, v);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(c.bar(B_Q_FULL));
+            }
             const int last_t = p.causal ? T - p.s_q + m_glob / p.H : T - 1;
+            const int full_end = p.causal ? T - p.s_q + 1 : T;  // tokens < full_end are visible to every row
             const int ntiles_req = (T + kPage - 1) / kPage;
             const int n = S.tile_end - S.tile_begin;
             float m_run = -INFINITY, l = 0.f;
             bool badpage = false;
-            bool alive = true;
             for (int jj = 0; jj < n; ++jj, ++it) {
                 const int tile = S.tile_begin + jj;
                 const int32_t page = p.block_table[(int64_t)S.b * p.max_pages + tile];
                 badpage |= !(page >= 0 && page < p.num_pages);
-                const int sb = it & 1;
-                alive = wait_bar(c, c.bar(B_S_FULL0 + sb), (it >> 1) & 1, false);
+                alive = wait_bar(c, c.bar(B_S_FULL0 + (it & 1)), (it >> 1) & 1);
                 if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
                 ptx::tc_fence_after();
-                uint32_t sr[64];
-                ptx::tmem_ld32(trow + kTmemS + 64u * sb, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                ptx::tmem_ld32(trow + kTmemS + 64u * sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                uint32_t sr[32];
+                ptx::tmem_ld16x32<32>(t_hi + kColS + 64u * (it & 1), sr);
                 ptx::tmem_wait_ld();
-                float s[64];
+                float s[32];
+                const float sc = p.score_scale_log2;
+                const int tok0 = tile * kPage + 32 * half;
+                if (tile * kPage + kPage <= full_end) {
 #pragma unroll
-                for (int k = 0; k < 64; ++k) s[k] = __uint_as_float(sr[k]);
-                // exchange partial scores with the peer CTA
-                if (it > 0) alive = wait_bar(c, c.bar(B_XEMPTY), (it - 1) & 1, true);
-                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
+                    for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(sr[k]) * sc;
+                } else {
 #pragma unroll
-                for (int k4 = 0; k4 < 16; ++k4)
-                    ptx::st_async_v4(xchg_remote + (uint32_t)(k4 * kRows + row) * 16u,
-                                     make_float4(s[4 * k4], s[4 * k4 + 1], s[4 * k4 + 2], s[4 * k4 + 3]), xfull_remote);
-                alive = wait_bar(c, c.bar(B_XFULL), it & 1, true);
-                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
-#pragma unroll
-                for (int k4 = 0; k4 < 16; ++k4) {
-                    const float4 v = *reinterpret_cast<const float4*>(xchg_f + (size_t)(k4 * kRows + row) * 4);
-                    s[4 * k4] += v.x;
-                    s[4 * k4 + 1] += v.y;
-                    s[4 * k4 + 2] += v.z;
-                    s[4 * k4 + 3] += v.w;
+                    for (int k = 0; k < 32; ++k) {
+                        const int t = tok0 + k;
+                        s[k] = (t < T && t <= last_t) ? __uint_as_float(sr[k]) * sc : -INFINITY;
+                    }
                 }
-                // all 128 rows have read the peer's data: re-arm and release the buffer
-                ptx::mbar_arrive(c.bar(B_SMSYNC));
-                alive = wait_bar(c, c.bar(B_SMSYNC), it & 1, false);
-                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
-                if (tid == 0) {
-                    ptx::mbar_arrive_expect_tx(c.bar(B_XFULL), kXchgBytes);
-                    ptx::mbar_arrive_remote(xempty_remote);
-                }
-                // base-2 scores with the visibility mask
-                const int tok0 = tile * kPage;
-                float mt = -INFINITY;
+                float mx[8];
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const int t = tok0 + k;
-                    s[k] = (t < T && t <= last_t) ? s[k] * p.score_scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, s[k]);
-                }
+                for (int k = 0; k < 8; ++k) mx[k] = fmaxf(fmaxf(s[4 * k], s[4 * k + 1]), fmaxf(s[4 * k + 2], s[4 * k + 3]));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
+                float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
                 const bool raise = mt > m_run + kRescaleThreshold;
                 float alpha = 1.f;
                 if (raise) {
@@ -406,67 +489,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (raise) m_run = mt;
                 if (__any_sync(0xffffffffu, need_o)) {
                     // O holds earlier pages of this split: wait for the last PV, rescale the rows
-                    alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1, false);
+                    alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1);
                     if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
                     ptx::tc_fence_after();
                     const float f = need_o ? alpha : 1.f;
 #pragma unroll 1
                     for (int q = 0; q < 8; ++q) {
                         uint32_t o[32];
-                        ptx::tmem_ld32(trow + kTmemO + 32 * q, o);
+                        ptx::tmem_ld16x32<32>(t_lo + 64u * q, o);
                         ptx::tmem_wait_ld();
 #pragma unroll
                         for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-                        ptx::tmem_st32(trow + kTmemO + 32 * q, o);
+                        ptx::tmem_st16x32<32>(t_lo + 64u * q, o);
                     }
                     ptx::tmem_wait_st();
                 }
-                uint32_t pk[32];
-                float rs = 0.f;
+                uint32_t pk[16];
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
+                const bool live = m_run != -INFINITY;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float p0 = m_run == -INFINITY ? 0.f : fast_exp2(s[2 * k] - m_run);
-                    const float p1 = m_run == -INFINITY ? 0.f : fast_exp2(s[2 * k + 1] - m_run);
-                    rs += p0 + p1;
+                for (int k = 0; k < 16; ++k) {
+                    const float p0 = live ? fast_exp2(s[2 * k] - m_run) : 0.f;
+                    const float p1 = live ? fast_exp2(s[2 * k + 1] - m_run) : 0.f;
+                    rs[k & 3] += p0 + p1;
                     pk[k] = pack_bf16(p0, p1);
                 }
-                l += rs;
+                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
                 if (tile == ntiles_req - 1 && (T % kPage) != 0) {
                     // rows past the request's end hold stale data (maybe NaN): zero their
                     // latent columns before the PV product reads them with P = 0
-                    alive = wait_bar(c, c.bar(B_KV_FULL0 + it % kStages), (it / kStages) & 1, false);
+                    alive = wait_bar(c, c.bar(B_KV_FULL0 + it % kStages), (it / kStages) & 1);
                     if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
                     const int r0 = T % kPage;
                     uint8_t* vb = smem + kOffKv + (it % kStages) * kStageBytes;
-                    const int pieces = (kPage - r0) * 4 * 8;  // rows x chunks x 16-byte pieces
+                    const int pieces = (kPage - r0) * 8 * 8;  // rows x latent chunks x 16-byte pieces
                     for (int q = tid; q < pieces; q += 128) {
-                        const int r = r0 + q / 32, j = (q / 8) % 4, w = q % 8;
-                        *reinterpret_cast<uint4*>(vb + j * kKvLatChunk + r * 128 + w * 16) = make_uint4(0, 0, 0, 0);
+                        const int r = r0 + q / 64, j = (q / 8) % 8, w = q % 8;
+                        *reinterpret_cast<uint4*>(vb + j * kChunk + r * 128 + w * 16) = make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();
                 }
-                ptx::tmem_st32(trow + kTmemS + 64u * sb, pk);
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(c.bar(B_P_READY0 + sb));
+                // the single P buffer is free once the previous page's PV has read it
+                if (jj > 0) {
+                    alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1);
+                    if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
+                }
+                {
+                    // P row `row`, tokens [32 half, 32 half + 32): four 16-byte chunks of the
+                    // 128-byte K-major row, 128-byte swizzle
+                    uint8_t* prow_s = pbuf + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int chunk = 4 * half + w;
+                        *reinterpret_cast<uint4*>(prow_s + ((chunk ^ (row & 7)) << 4)) =
+                            make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(c.bar(B_P_READY0 + (it & 1)));
             }
             if (!alive || *c.abort) break;
-            // epilogue: wait for the last PV of the split
-            alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1, false);
+            // epilogue: wait for the last PV of the split; the row sum is the two halves' sum
+            alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1);
             if (__any_sync(0xffffffffu, !alive)) break;
             ptx::tc_fence_after();
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
             if (badpage && tid == 0) set_status(h, kStatusOob, S.b);
             const float nanv = __int_as_float(0x7fc00000);
             const float inv = badpage ? nanv : (l > 0.f ? p.out_scale / l : 0.f);
 #pragma unroll 1
             for (int q = 0; q < 8; ++q) {
                 uint32_t o[32];
-                ptx::tmem_ld32(trow + kTmemO + 32 * q, o);
+                ptx::tmem_ld16x32<32>(t_lo + 64u * q, o);
                 ptx::tmem_wait_ld();
                 if (!row_valid) continue;
+                const int col = 64 * q + 32 * half;
                 if (!S.split) {
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * kDv +
-                                                          256 * crank + 32 * q);
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * kDv + col);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 w;
@@ -477,23 +576,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         dst[v] = w;
                     }
                 } else {
-                    float4* dst = reinterpret_cast<float4*>(po + prow * kDv + 256 * crank + 32 * q);
+                    float4* dst = reinterpret_cast<float4*>(po + prow * kDv + col);
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
                         dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
                                              __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
                 }
             }
-            if (row_valid && crank == 0) {
+            if (row_valid && half == 0) {
                 const float lse2 = badpage ? nanv : (l > 0.f ? m_run + __log2f(l) : -INFINITY);
                 if (!S.split)
                     p.lse[orow] = lse2 * kLn2;
                 else
                     plse[prow] = lse2;
             }
+            // the next split's q overwrites TMEM only after this epilogue's reads (same threads)
             ptx::tc_fence_before();
-            ptx::mbar_arrive(c.bar(B_O_EMPTY));
-            ++nseg;
         }
     }
 
@@ -501,7 +599,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
-    ptx::cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
 }
 
 // ------------------------------------------------------------------ host side
@@ -533,46 +630,49 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
 
 }  // namespace
 
-int sm100_pair_slots() {
-    // How many pairs of this kernel the current device runs at once (1 CTA per SM).
+int sm100_cta_slots() {
+    // CTAs of the scan kernel the current device keeps resident at once (one per SM).
     static int cached[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     if (dev < 64 && cached[dev] > 0) return cached[dev];
-    if (cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(decode_sm100_kernel<MLA_KV_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess)
         return -1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_sm100_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_sm100_kernel<MLA_KV_E4M3>, kThreadsE4m3,
+                                                      kSmemBytes) !=
+            cudaSuccess ||
+        per_sm <= 0)
+        return -1;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    const int n = per_sm * sms;
     if (dev < 64) cached[dev] = n;
     return n;
 }
 
-mla_status launch_decode_sm100(const DecodeParams& p, cudaStream_t stream) {
+template <int KV>
+mla_status launch_typed(const DecodeParams& p, cudaStream_t stream) {
     Sm100Args a;
     memset(&a, 0, sizeof(a));
     a.p = p;
-    const uint64_t qrows = (uint64_t)p.B * p.M;
     const uint64_t kvrows = (uint64_t)p.num_pages * kPage;
-    if (!make_map_2d(&a.tm_q_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, kDqk, qrows, kDqk * 2, 64, kRows,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&a.tm_q_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, kDqk, qrows, kDqk * 2, 32, kRows,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_2d(&a.tm_kv_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 64, kTok,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&a.tm_kv_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 32, kTok,
-                     CU_TENSOR_MAP_SWIZZLE_64B))
-        return MLA_ERR_CUDA;
-    if (cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+    const bool ok = KV == MLA_KV_E4M3
+                        ? make_map_2d(&a.tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.kv, kDqk, kvrows, kDqk, 64, kTok,
+                                      CU_TENSOR_MAP_SWIZZLE_NONE)
+                        : make_map_2d(&a.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 64,
+                                      kTok, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return MLA_ERR_CUDA;
+    if (cudaFuncSetAttribute(decode_sm100_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
         cudaSuccess)
         return MLA_ERR_CUDA;
-    const int clusters = p.groups_launched * num_row_blocks(p.s_q, p.H);
-    decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(a);
+    const int ctas = p.groups_launched * num_row_blocks(p.s_q, p.H);
+    decode_sm100_kernel<KV><<<ctas, threads_for<KV>(), kSmemBytes, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status launch_decode_sm100(const DecodeParams& p, int kv_dtype, cudaStream_t stream) {
+    return kv_dtype == MLA_KV_E4M3 ? launch_typed<MLA_KV_E4M3>(p, stream) : launch_typed<MLA_KV_BF16>(p, stream);
 }
 
 }  // namespace mla

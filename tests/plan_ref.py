@@ -12,7 +12,7 @@ PAGE = 64
 
 
 def num_groups_for(num_sms, nqb):
-    return max(1, (num_sms // 2) // nqb)
+    return max(1, num_sms // nqb)
 
 
 def plan(seq_lens, G):

@@ -82,7 +82,7 @@ def test_decode_rejects_bad_arguments_before_any_launch(kw, code):
 def test_plan_rejects_bad_arguments():
     assert _abi.mla_decode_plan(None, 2, 4, 16, 148, 256, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
     assert _abi.mla_decode_plan(16, 2, 4, 16, 148, 256, 1024, None) == _abi.MLA_ERR_WORKSPACE_TOO_SMALL
-    assert _abi.mla_decode_plan(16, 2, 4, 16, 1, 256, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_decode_plan(16, 2, 4, 16, -1, 256, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
     assert _abi.mla_decode_plan(16, 2, 4, 16, 148, 300, 1 << 30, None) == _abi.MLA_ERR_INVALID_ARG
 
 
