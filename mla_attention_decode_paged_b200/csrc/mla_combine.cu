@@ -7,99 +7,129 @@
 // the reduction pass of split-KV decoding ["Faster kernels, slower engine", 7.1 Gluon
 // MLA decode].  A split in which a row sees no token has lse2_j = -inf and o_j = 0, so
 // it drops out.  The kernel reads every partial once; it is bound by that read.
+#include <string.h>
+
 #include "mla_common.cuh"
 
 namespace mla {
 
-constexpr int kCombineThreads = 512;  // 4 groups of 128 threads; a thread owns one float4 column
-constexpr int kCombineMaxSplits = kMaxGroups + 1;
+constexpr int kCombineThreads = 256;  // 16 rows x 16 column quads
+constexpr int kWChunk = 64;           // splits whose weights are in shared memory at once
+constexpr int kPre = 8;               // partials loaded before the weights are known
 
-// grid (B, nqb, 64): one folded row per CTA.  The row's split weights are computed once
-// into shared memory; group j of the CTA accumulates the splits j, j+4, j+8, ... for its
-// float4 column (several independent loads in flight per thread), and the four group
-// sums are added through shared memory.
+// grid (B, 4 nqb, 8): one CTA per (request, 16-row group, 64 columns).  Thread t owns row
+// t % 16 and column quad t / 16 of the tile; in the workspace's quad-interleaved partial
+// layout the CTA's tile of one split is 4 KB contiguous, read by the 256 threads with
+// one 16-byte load each.  The first kPre partials are loaded before the weights are
+// computed, so their latency overlaps that computation.
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __restrict__ ws, int B, int s_q, int H,
                                                                   __nv_bfloat16* __restrict__ out,
                                                                   float* __restrict__ lse) {
-    __shared__ float wsh[kCombineMaxSplits];
-    __shared__ float4 part[3][128];
-    __shared__ float red[2];
+    __shared__ float wsh[kWChunk][16];
+    __shared__ float Lsh[16], Msh[16];
     const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
+    // launched as a programmatic dependent of the scan: nothing is read before it completes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
-    const int b = blockIdx.x, qb = blockIdx.y, r = blockIdx.z;
+    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3, c64 = blockIdx.z;
     const int M = s_q * H;
-    const int row = qb * kRowsPerBlock + r;
-    if (row >= M) return;
+    const int row0 = qb * kRowsPerBlock + g * 16;
+    if (row0 >= M) return;
     const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
     const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
     if (ns <= 1) return;  // written directly by the decode kernel
     const int nqb = h->nqb;
-    const float* plse = ws_ptr<float>(ws, h->off_plse);
-    const float* po = ws_ptr<float>(ws, h->off_po);
-    const int64_t stride = (int64_t)nqb * kRowsPerBlock;  // rows between consecutive segments
-    const int64_t prow0 = ((int64_t)s0 * nqb + qb) * kRowsPerBlock + r;
-    const int tid = threadIdx.x, grp = tid >> 7, c4 = tid & 127;
+    const int tid = threadIdx.x, r16 = tid & 15, cq = tid >> 4;
+    // split j: partial tile at pbase + j * jstride (float4), lse2 of row r at lbase[j * lstride + r]
+    const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
+                          ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + (16 * c64 + cq) * 16 + r16;
+    const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
+    const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
+    const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
 
-    // L = log2 sum_j 2^lse2_j and the weights 2^(lse2_j - L), by warp 0
-    if (tid < 32) {
-        float mx = -INFINITY;
-        for (int j = tid; j < ns; j += 32) mx = fmaxf(mx, plse[prow0 + j * stride]);
+    float4 v[kPre];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int u = 0; u < kPre; ++u) v[u] = u < ns ? pbase[u * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // L = log2 sum_j 2^lse2_j per row: warp w takes rows 2w and 2w + 1 (one per half-warp)
+    {
+        const int lane = tid & 31, r = 2 * (tid >> 5) + (lane >> 4), k = lane & 15;
+        float mx = -INFINITY;
+        for (int j = k; j < ns; j += 16) mx = fmaxf(mx, lbase[j * lstride + r]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sum = 0.f;
         if (mx != -INFINITY)
-            for (int j = tid; j < ns; j += 32) sum += fast_exp2(plse[prow0 + j * stride] - mx);
+            for (int j = k; j < ns; j += 16) sum += fast_exp2(lbase[j * lstride + r] - mx);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const float L = mx + __log2f(sum);
-        for (int j = tid; j < ns && j < kCombineMaxSplits; j += 32) {
-            const float l2 = plse[prow0 + j * stride];
-            wsh[j] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - L);  // an empty split drops out
-        }
-        if (tid == 0) {
-            red[0] = L;
-            red[1] = mx;
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (k == 0) {
+            Lsh[r] = mx + __log2f(sum);
+            Msh[r] = mx;
         }
     }
     __syncthreads();
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int j = grp;
-    for (; j + 12 < ns; j += 16) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = reinterpret_cast<const float4*>(po + (prow0 + (int64_t)(j + 4 * u) * stride) * kDv)[c4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float w = wsh[j + 4 * u];
-            acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+    for (int j0 = 0; j0 < ns; j0 += kWChunk) {
+        const int nj = min(kWChunk, ns - j0);
+        for (int e = tid; e < nj * 16; e += kCombineThreads) {
+            const int jj = e >> 4, r = e & 15;
+            const float l2 = lbase[(int64_t)(j0 + jj) * lstride + r];
+            wsh[jj][r] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - Lsh[r]);  // an empty split drops out
         }
-    }
-    for (; j < ns; j += 4) {
-        const float4 v = reinterpret_cast<const float4*>(po + (prow0 + (int64_t)j * stride) * kDv)[c4];
-        const float w = wsh[j];
-        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
-    }
-    if (grp > 0) part[grp - 1][c4] = acc;
-    __syncthreads();
-    if (grp == 0) {
+        __syncthreads();
+        int jj = 0;
+        if (j0 == 0) {
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const float4 v = part[k][c4];
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            for (int u = 0; u < kPre; ++u) {
+                const float w = u < nj ? wsh[u][r16] : 0.f;
+                acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+            }
+            jj = kPre;
         }
+        for (; jj + 3 < nj; jj += 4) {
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = pbase[(j0 + jj + u) * jstride];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float w = wsh[jj + u][r16];
+                acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
+            }
+        }
+        for (; jj < nj; ++jj) {
+            const float4 x = pbase[(j0 + jj) * jstride];
+            const float w = wsh[jj][r16];
+            acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+        }
+        __syncthreads();
+    }
+    const int m = row0 + r16;
+    if (m < M) {
         __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
         __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
         uint2 pk;
         pk.x = *reinterpret_cast<uint32_t*>(&lo);
         pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDv + 4 * c4) = pk;
-        if (c4 == 0) lse[(int64_t)b * M + row] = (red[1] == -INFINITY) ? -INFINITY : red[0] * kLn2;
+        *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) = pk;
+        if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
     }
 }
 
 mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream) {
-    dim3 grid(B, num_row_blocks(s_q, H), kRowsPerBlock);
-    combine_kernel<<<grid, kCombineThreads, 0, stream>>>(ws, B, s_q, H, reinterpret_cast<__nv_bfloat16*>(out), lse);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(B, 4 * num_row_blocks(s_q, H), kDv / 64);
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel, ws, B, s_q, H, reinterpret_cast<__nv_bfloat16*>(out), lse) !=
+        cudaSuccess)
+        return MLA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -48,7 +48,10 @@ struct __align__(16) PlanHeader {
     int64_t off_req_seg;      // int32 [B + 1]
     int64_t off_segs;         // Segment [max_segments]
     int64_t off_plse;         // float [max_segments][nqb][64]   (log2 domain)
-    int64_t off_po;           // float [max_segments][nqb][64][512]
+    int64_t off_po;           // float [max_segments][nqb][4][128][16][4]: per 16-row group of a
+                              // 64-row block, column quads outermost, the group's 16 rows next,
+                              // the quad's 4 columns innermost (row r, column c of the block at
+                              // (r / 16) * 8192 + (c / 4) * 64 + (r % 16) * 4 + c % 4)
     int64_t total_bytes;
 };
 

@@ -20,7 +20,9 @@
 //       output scales.
 //   MMA (one thread): S = q . K^T with q read from TMEM (M=64 N=64, 36 K-steps), then
 //       O += P . V with P (bf16) and V (the same page, read MN-major) from shared memory
-//       (M=64 N=256, twice, 4 K-steps each).
+//       (M=64 N=256, twice, 4 K-steps each).  P is written over the page's rope chunk,
+//       which only the score MMAs read: every stage carries its own P, and the softmax
+//       of a page never waits for the previous page's PV.
 //   softmax (4 warps, 16 rows each, two threads per row with 32 scores each): base-2
 //       online softmax with the causal draft mask; the running max is only raised (and
 //       O rescaled) when a score exceeds it by more than 8, so P <= 256.
@@ -53,11 +55,14 @@ constexpr uint32_t kChunk = kTok * 128;              // 64 tokens x 64 columns b
 constexpr uint32_t kStageBytes = 9 * kChunk;         // 8 latent chunks + 1 rope chunk: 72 KB
 constexpr uint32_t kRawChunk = kTok * 64;            // e4m3: 64 tokens x 64 columns, in the upper half
 constexpr uint32_t kRawStageBytes = 9 * kRawChunk;   //        of each bf16 chunk slot
-constexpr uint32_t kPBytes = kRows * kTok * 2;       // P: 64 rows x 64 tokens bf16
 constexpr uint32_t kOffKv = 0;
-constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffP + kPBytes;
+constexpr uint32_t kOffPInStage = 8 * kChunk;        // P (64 rows x 64 tokens bf16) over the rope chunk
+constexpr uint32_t kOffEpi = kOffKv + kStages * kStageBytes;  // epilogue staging: 2 KB per softmax warp
+constexpr uint32_t kEpiWarpBytes = 16 * 128;
+constexpr uint32_t kOffBar = kOffEpi + 4 * kEpiWarpBytes;
+static_assert(kRows * kTok * 2 == kChunk, "P fills the rope chunk exactly");
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+static_assert(kSmemBytes <= 232448, "dynamic shared memory limit per block");
 
 enum : int {
     B_KV_FULL0 = 0, B_KV_EMPTY0 = B_KV_FULL0 + kStages, B_Q_FULL = B_KV_EMPTY0 + kStages, B_S_FULL0,
@@ -165,6 +170,11 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
     const DecodeParams& p = args.p;
     PlanHeader* h = reinterpret_cast<PlanHeader*>(p.ws);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the combine may start its prologue now; it waits for this grid before reading
+    ptx::griddep_launch_dependents();
+    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
+    // the plan (and every earlier write) must be complete before the header is read
+    ptx::griddep_wait();
 
     if (h->magic != kPlanMagic || h->B != p.B || h->s_q != p.s_q || h->H != p.H ||
         h->num_groups > p.groups_launched) {
@@ -197,7 +207,6 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
         ptx::mbar_init(c.bar(B_DRAIN), 1);
         ptx::fence_mbar_init_cluster();
     }
-    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
     if (warp == 1) {
         ptx::tmem_alloc(sbase + kOffTmemHolder, kTmemCols);
         ptx::tmem_relinquish();
@@ -213,50 +222,60 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int it = 0;
-            for (int si = seg_lo; si < seg_hi && !*c.abort; ++si) {
-                const Segment S = segs[si];
-                const int T = p.seq_lens[S.b];
-                if (!request_ok(p, T)) continue;
-                bool ok = true;
-                for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
+        // The whole warp walks the tiles; every 32 tiles each lane fetches one block-table
+        // entry, so the page ids reach lane 0 (which waits and issues) by shuffles instead
+        // of one dependent global load per page.
+        int it = 0;
+        bool ok = true;
+        for (int si = seg_lo; si < seg_hi && ok; ++si) {
+            if (__shfl_sync(0xffffffffu, lane == 0 ? *c.abort : 0, 0)) break;
+            const Segment S = segs[si];
+            const int T = p.seq_lens[S.b];
+            if (!request_ok(p, T)) continue;
+            const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
+            int32_t pg = 0;
+            for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
+                const int j = (t - S.tile_begin) & 31;
+                if (j == 0) pg = (t + lane < S.tile_end) ? bt_row[t + lane] : 0;
+                const int32_t page = __shfl_sync(0xffffffffu, pg, j);
+                if (lane == 0) {
                     const int st = it % kStages;
                     if (it >= kStages && !wait_bar(c, c.bar(B_KV_EMPTY0 + st), ((it / kStages) - 1) & 1)) {
                         ok = false;
-                        break;
-                    }
-                    const int32_t page = p.block_table[(int64_t)S.b * p.max_pages + t];
-                    // an invalid page id becomes a box entirely out of range (zero fill); the
-                    // softmax warps see the same id and poison the request's rows
-                    const int ky = (page >= 0 && page < p.num_pages) ? page * kPage : -kPage;
-                    const uint32_t dst = sbase + kOffKv + st * kStageBytes;
-                    if (kE4m3) {
-                        ptx::mbar_arrive_expect_tx(c.bar(B_RAW0 + st), kRawStageBytes);
-#pragma unroll
-                        for (int j = 0; j < 9; ++j)
-                            ptx::tma_load_2d(dst + j * kChunk + kRawChunk, &args.tm_kv, c.bar(B_RAW0 + st), 64 * j, ky);
                     } else {
-                        ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
+                        // an invalid page id becomes a box entirely out of range (zero fill);
+                        // the softmax warps see the same id and poison the request's rows
+                        const int ky = (page >= 0 && page < p.num_pages) ? page * kPage : -kPage;
+                        const uint32_t dst = sbase + kOffKv + st * kStageBytes;
+                        if (kE4m3) {
+                            ptx::mbar_arrive_expect_tx(c.bar(B_RAW0 + st), kRawStageBytes);
 #pragma unroll
-                        for (int j = 0; j < 9; ++j)
-                            ptx::tma_load_2d(dst + j * kChunk, &args.tm_kv, c.bar(B_KV_FULL0 + st), 64 * j, ky);
+                            for (int jb = 0; jb < 9; ++jb)
+                                ptx::tma_load_2d(dst + jb * kChunk + kRawChunk, &args.tm_kv, c.bar(B_RAW0 + st),
+                                                 64 * jb, ky);
+                        } else {
+                            ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
+#pragma unroll
+                            for (int jb = 0; jb < 9; ++jb)
+                                ptx::tma_load_2d(dst + jb * kChunk, &args.tm_kv, c.bar(B_KV_FULL0 + st), 64 * jb,
+                                                 ky);
+                        }
                     }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
-            if (*c.abort) {
-                for (int k = (it > kStages ? it - kStages : 0); k < it; ++k)
-                    drain_wait(c.bar((kE4m3 ? B_RAW0 : B_KV_FULL0) + k % kStages), (k / kStages) & 1);
-            }
+        }
+        if (lane == 0 && *c.abort) {
+            for (int k = (it > kStages ? it - kStages : 0); k < it; ++k)
+                drain_wait(c.bar((kE4m3 ? B_RAW0 : B_KV_FULL0) + k % kStages), (k / kStages) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // An event loop: the score MMAs of the next page and the PV MMAs of the oldest
-        // page whose P is ready are issued in whichever order their inputs arrive, so a
-        // stage is released as soon as its PV completes instead of waiting behind the
-        // next page's load.  The tensor core runs them in issue order.  Barriers are
-        // polled with test_wait, which never suspends the thread.
+        // page whose P is ready are issued in whichever order their inputs arrive.  The
+        // tensor core runs them in issue order.  Barriers are polled with test_wait, which
+        // never suspends the thread.
         if (lane == 0) {
             int it = 0, nseg = 0;
             bool ok = true;
@@ -272,7 +291,9 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 uint32_t spins = 0;
                 while (npv < n) {
                     bool progressed = false;
-                    // S(ns) reuses the score buffer of page ns-2, whose PV must be issued first
+                    // S(ns) reuses the score buffer of page ns-2, whose PV must be issued first.
+                    // A score chain is issued whole: PV MMAs placed between its K-steps (another
+                    // accumulator) slow the chain down far more than they gain.
                     if (ns < n && ns <= npv + 1) {
                         const int its = it + ns, st = its % kStages;
                         if (ptx::mbar_test_wait(c.bar(B_KV_FULL0 + st), (its / kStages) & 1)) {
@@ -298,9 +319,9 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                             const bool first = npv == 0;
                             // A = P (K-major); B = V, MN-major: 64-column blocks 8 KB apart (leading
                             // offset), 8-token groups 1 KB apart (stride offset)
-                            const uint64_t a0 = ptx::smem_desc(sbase + kOffP, 16, 1024, ptx::kSwizzle128);
-                            const uint64_t v0 = ptx::smem_desc(sbase + kOffKv + (itp % kStages) * kStageBytes, kChunk,
-                                                               1024, ptx::kSwizzle128);
+                            const uint32_t stage = sbase + kOffKv + (itp % kStages) * kStageBytes;
+                            const uint64_t a0 = ptx::smem_desc(stage + kOffPInStage, 16, 1024, ptx::kSwizzle128);
+                            const uint64_t v0 = ptx::smem_desc(stage, kChunk, 1024, ptx::kSwizzle128);
 #pragma unroll
                             for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -396,7 +417,6 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
         const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(p.q);
         float* plse = ws_ptr<float>(p.ws, h->off_plse);
         float* po = ws_ptr<float>(p.ws, h->off_po);
-        uint8_t* pbuf = smem + kOffP;
         int it = 0;
         bool alive = true;
 
@@ -414,30 +434,42 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                         for (int k = 0; k < 256; ++k) dst[k] = __float2bfloat16_rn(nanv);
                         if (half == 0) p.lse[orow] = nanv;
                     } else {
-                        float* dst = po + prow * kDv + 256 * half;
-                        for (int k = 0; k < 256; ++k) dst[k] = nanv;
+                        // the row's columns [256 half, +256) in the quad-interleaved partial layout
+                        float* blk = po + ((int64_t)si * nqb + qb) * kRows * kDv + (row >> 4) * 8192 + (row & 15) * 4;
+                        for (int k = 0; k < 256; ++k) {
+                            const int col = 256 * half + k;
+                            blk[(col >> 2) * 64 + (col & 3)] = nanv;
+                        }
                         if (half == 0) plse[prow] = nanv;
                     }
                 }
                 continue;
             }
             if (*c.abort) break;
-            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row
+            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row,
+            // loaded three column blocks at a time (three memory round trips, not nine)
             {
                 const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + m_glob) * kDqk);
 #pragma unroll 1
-                for (int k = 0; k < 9; ++k) {
-                    uint32_t v[16];
-                    const int d0 = 64 * k + 32 * half;  // first of this thread's 32 dims
+                for (int kb = 0; kb < 9; kb += 3) {
+                    uint4 x[3][4];
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const uint4 x = row_valid ? src[d0 / 8 + w] : make_uint4(0, 0, 0, 0);
-                        v[4 * w] = x.x;
-                        v[4 * w + 1] = x.y;
-                        v[4 * w + 2] = x.z;
-                        v[4 * w + 3] = x.w;
+                    for (int k = 0; k < 3; ++k)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)  // dims [64 (kb + k) + 32 half, +32)
+                            x[k][w] = row_valid ? src[(64 * (kb + k) + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        uint32_t v[16];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            v[4 * w] = x[k][w].x;
+                            v[4 * w + 1] = x[k][w].y;
+                            v[4 * w + 2] = x[k][w].z;
+                            v[4 * w + 3] = x[k][w].w;
+                        }
+                        ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * (kb + k), v);
                     }
-                    ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * k, v);
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
@@ -529,14 +561,11 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                     }
                     ptx::fence_proxy_async_smem();
                 }
-                // the single P buffer is free once the previous page's PV has read it
-                if (jj > 0) {
-                    alive = wait_bar(c, c.bar(B_PV_DONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1);
-                    if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
-                }
                 {
                     // P row `row`, tokens [32 half, 32 half + 32): four 16-byte chunks of the
-                    // 128-byte K-major row, 128-byte swizzle
+                    // 128-byte K-major row, 128-byte swizzle, over the page's rope chunk (the
+                    // score MMAs that read it have completed: S_FULL was waited above)
+                    uint8_t* pbuf = smem + kOffKv + (it % kStages) * kStageBytes + kOffPInStage;
                     uint8_t* prow_s = pbuf + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
@@ -546,6 +575,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                     }
                 }
                 ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();  // the score loads above precede the MMAs that follow P_READY
                 ptx::mbar_arrive(c.bar(B_P_READY0 + (it & 1)));
             }
             if (!alive || *c.abort) break;
@@ -557,30 +587,51 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             if (badpage && tid == 0) set_status(h, kStatusOob, S.b);
             const float nanv = __int_as_float(0x7fc00000);
             const float inv = badpage ? nanv : (l > 0.f ? p.out_scale / l : 0.f);
-#pragma unroll 1
-            for (int q = 0; q < 8; ++q) {
-                uint32_t o[32];
-                ptx::tmem_ld16x32<32>(t_lo + 64u * q, o);
-                ptx::tmem_wait_ld();
-                if (!row_valid) continue;
-                const int col = 64 * q + 32 * half;
-                if (!S.split) {
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * kDv + col);
+            // O / l.  A split writes its fp32 partial in the workspace's quad-interleaved layout
+            // (column quads outermost, then the warp's 16 rows): each store instruction of the
+            // warp covers two whole 256-byte runs.  A request held whole goes to the bf16
+            // output, row-major, through a 2 KB staging tile per warp (16 rows x 128 bytes,
+            // 16-byte pieces XOR-swizzled by row) so that every store writes whole row segments.
+            uint8_t* stg = smem + kOffEpi + (warp - 2) * kEpiWarpBytes;
+            const int rows_ok = min(16, p.M - (qb * kRows + quad * 16));  // valid rows of this warp
+            const int64_t out_row0 = (int64_t)S.b * p.M + qb * kRows + quad * 16;
+            float4* pq = reinterpret_cast<float4*>(po + ((int64_t)si * nqb + qb) * kRows * kDv) + quad * 2048 +
+                         8 * half * 16 + r16;  // + (16 q + v) * 16 for columns 64 q + 32 half + 4 v
+            uint32_t o[2][32];
+            ptx::tmem_ld16x32<32>(t_lo, o[0]);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-                        dst[v] = w;
+            for (int q = 0; q < 8; ++q) {
+                // the next chunk's TMEM load is in flight while this one is stored
+                ptx::tmem_wait_ld();
+                if (q + 1 < 8) ptx::tmem_ld16x32<32>(t_lo + 64u * (q + 1), o[(q + 1) & 1]);
+                const uint32_t* oq = o[q & 1];
+                if (!S.split) {
+                    // bf16: the row's 64 columns are 8 pieces; this thread holds pieces 4 half + w
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(oq[8 * w + 0]) * inv, __uint_as_float(oq[8 * w + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(oq[8 * w + 2]) * inv, __uint_as_float(oq[8 * w + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(oq[8 * w + 4]) * inv, __uint_as_float(oq[8 * w + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(oq[8 * w + 6]) * inv, __uint_as_float(oq[8 * w + 7]) * inv);
+                        *reinterpret_cast<uint4*>(stg + r16 * 128 + (((4 * half + w) ^ (r16 & 7)) << 4)) = v;
                     }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(po + prow * kDv + col);
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int idx = lane + 32 * j, rr = idx >> 3, w = idx & 7;
+                        const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((w ^ (rr & 7)) << 4));
+                        if (rr < rows_ok)
+                            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                      (out_row0 + rr) * kDv + 64 * q + 8 * w) = v;
+                    }
+                    __syncwarp();
+                } else if (row_valid) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
-                        dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                             __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                        pq[(16 * q + v) * 16] =
+                            make_float4(__uint_as_float(oq[4 * v]) * inv, __uint_as_float(oq[4 * v + 1]) * inv,
+                                        __uint_as_float(oq[4 * v + 2]) * inv, __uint_as_float(oq[4 * v + 3]) * inv);
                 }
             }
             if (row_valid && half == 0) {
@@ -667,7 +718,20 @@ mla_status launch_typed(const DecodeParams& p, cudaStream_t stream) {
         cudaSuccess)
         return MLA_ERR_CUDA;
     const int ctas = p.groups_launched * num_row_blocks(p.s_q, p.H);
-    decode_sm100_kernel<KV><<<ctas, threads_for<KV>(), kSmemBytes, stream>>>(a);
+    // programmatic dependent launch: the prologue (barriers, TMEM, tensor map) overlaps the
+    // tail of the previous grid in the stream; the kernel waits for it before any global access
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(threads_for<KV>());
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_sm100_kernel<KV>, a) != cudaSuccess) return MLA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

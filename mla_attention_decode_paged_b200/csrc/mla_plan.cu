@@ -91,6 +91,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     int32_t* req_seg = ws_ptr<int32_t>(ws, L.off_req_seg);
     Segment* segs = ws_ptr<Segment>(ws, L.off_segs);
     const int tid = threadIdx.x;
+    // the scan kernel (a programmatic dependent) may start its prologue; it waits for this
+    // grid to complete before reading the plan
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (tid == 0) bad_first = B;
     __syncthreads();
