@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         // The whole warp walks the tiles; every 32 tiles each lane fetches one block-table
-        // entry, so the page ids reach lane 0 (which waits and issues) by shuffles instead
-        // of one dependent global load per page.
+        // entry (one window ahead), so the page ids reach lane 0 (which waits and issues) by
+        // shuffles instead of one dependent global load per page.
         int it = 0;
         bool ok = true;
         for (int si = seg_lo; si < seg_hi && ok; ++si) {
@@ -233,10 +233,13 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             const int T = p.seq_lens[S.b];
             if (!request_ok(p, T)) continue;
             const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
-            int32_t pg = 0;
+            int32_t pg = 0, pgn = 0;  // page ids of tiles [t0, t0 + 32) and [t0 + 32, t0 + 64)
             for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
                 const int j = (t - S.tile_begin) & 31;
-                if (j == 0) pg = (t + lane < S.tile_end) ? bt_row[t + lane] : 0;
+                if (j == 0) {
+                    pg = t == S.tile_begin ? ((t + lane < S.tile_end) ? bt_row[t + lane] : 0) : pgn;
+                    pgn = (t + 32 + lane < S.tile_end) ? bt_row[t + 32 + lane] : 0;
+                }
                 const int32_t page = __shfl_sync(0xffffffffu, pg, j);
                 if (lane == 0) {
                     const int st = it % kStages;
@@ -446,20 +449,24 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 continue;
             }
             if (*c.abort) break;
-            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row,
-            // loaded three column blocks at a time (three memory round trips, not nine)
+            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row.
+            // The loads of a batch are all issued before the first is used: at a split's start
+            // the memory system is full of the first pages' loads, and every dependent round
+            // trip here delays the first score MMA.  One batch of 36 loads per thread; three
+            // for an e4m3 cache, whose kernel has fewer registers per thread.
             {
+                constexpr int kQBatch = kE4m3 ? 3 : 9;  // column blocks per batch
                 const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + m_glob) * kDqk);
 #pragma unroll 1
-                for (int kb = 0; kb < 9; kb += 3) {
-                    uint4 x[3][4];
+                for (int kb = 0; kb < 9; kb += kQBatch) {
+                    uint4 x[kQBatch][4];
 #pragma unroll
-                    for (int k = 0; k < 3; ++k)
+                    for (int k = 0; k < kQBatch; ++k)
 #pragma unroll
                         for (int w = 0; w < 4; ++w)  // dims [64 (kb + k) + 32 half, +32)
                             x[k][w] = row_valid ? src[(64 * (kb + k) + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int k = 0; k < 3; ++k) {
+                    for (int k = 0; k < kQBatch; ++k) {
                         uint32_t v[16];
 #pragma unroll
                         for (int w = 0; w < 4; ++w) {
@@ -597,14 +604,8 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             const int64_t out_row0 = (int64_t)S.b * p.M + qb * kRows + quad * 16;
             float4* pq = reinterpret_cast<float4*>(po + ((int64_t)si * nqb + qb) * kRows * kDv) + quad * 2048 +
                          8 * half * 16 + r16;  // + (16 q + v) * 16 for columns 64 q + 32 half + 4 v
-            uint32_t o[2][32];
-            ptx::tmem_ld16x32<32>(t_lo, o[0]);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                // the next chunk's TMEM load is in flight while this one is stored
-                ptx::tmem_wait_ld();
-                if (q + 1 < 8) ptx::tmem_ld16x32<32>(t_lo + 64u * (q + 1), o[(q + 1) & 1]);
-                const uint32_t* oq = o[q & 1];
+            // one column chunk (64 columns) of O / l from registers to memory
+            auto store_chunk = [&](int q, const uint32_t(&oq)[32]) {
                 if (!S.split) {
                     // bf16: the row's 64 columns are 8 pieces; this thread holds pieces 4 half + w
 #pragma unroll
@@ -633,6 +634,20 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                             make_float4(__uint_as_float(oq[4 * v]) * inv, __uint_as_float(oq[4 * v + 1]) * inv,
                                         __uint_as_float(oq[4 * v + 2]) * inv, __uint_as_float(oq[4 * v + 3]) * inv);
                 }
+            };
+            // two register sets: the next chunk's TMEM load is in flight while one is stored.
+            // The loop is not unrolled: this code runs once per split, from a cold
+            // instruction cache, so its size costs more than its loop overhead.
+            uint32_t oa[32], ob[32];
+            ptx::tmem_ld16x32<32>(t_lo, oa);
+#pragma unroll 1
+            for (int q = 0; q < 8; q += 2) {
+                ptx::tmem_wait_ld();
+                ptx::tmem_ld16x32<32>(t_lo + 64u * (q + 1), ob);
+                store_chunk(q, oa);
+                ptx::tmem_wait_ld();
+                if (q + 2 < 8) ptx::tmem_ld16x32<32>(t_lo + 64u * (q + 2), oa);
+                store_chunk(q + 1, ob);
             }
             if (row_valid && half == 0) {
                 const float lse2 = badpage ? nanv : (l > 0.f ? m_run + __log2f(l) : -INFINITY);

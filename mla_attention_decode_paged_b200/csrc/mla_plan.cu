@@ -20,37 +20,39 @@ constexpr int kPlanThreads = 256;
 // In-place exclusive prefix sum of a[0..n) by the whole block (n + 1 entries are written:
 // a[n] receives the total).  Each thread scans a contiguous chunk; the chunk totals are
 // scanned with warp shuffles (one warp per 32 chunks, then one warp over the 8 warp sums).
-template <typename T>
-__device__ void block_exclusive_scan(T* a, int n, T* partial) {
+// The caller synchronises the block before the call; the call ends with a barrier.  Not
+// inlined: the plan runs once per launch on a cold SM, so one shared copy of the code
+// costs fewer instruction fetches than three inlined ones.
+__device__ __noinline__ void block_exclusive_scan(int64_t* a, int n, int64_t* partial) {
     static_assert(kPlanThreads == 256, "two-level warp scan below assumes 8 warps");
     const int per = (n + kPlanThreads - 1) / kPlanThreads;
     const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    T run = 0;
+    int64_t run = 0;
     for (int i = lo; i < hi; ++i) run += a[i];
     // inclusive scan of the chunk totals within the warp
-    T v = run;
+    int64_t v = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const T u = __shfl_up_sync(0xffffffffu, v, o);
+        const int64_t u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
     }
     if (lane == 31) partial[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        T w = lane < 8 ? partial[lane] : 0;
+        int64_t w = lane < 8 ? partial[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 8; o <<= 1) {
-            const T u = __shfl_up_sync(0xffffffffu, w, o);
+            const int64_t u = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) w += u;
         }
         if (lane < 8) partial[8 + lane] = w;  // inclusive totals of warps 0..lane
     }
     __syncthreads();
-    T acc = (v - run) + (warp > 0 ? partial[8 + warp - 1] : 0);  // exclusive offset of this chunk
+    int64_t acc = (v - run) + (warp > 0 ? partial[8 + warp - 1] : 0);  // exclusive offset of this chunk
     if (threadIdx.x == kPlanThreads - 1) a[n] = partial[15];
     for (int i = lo; i < hi; ++i) {
-        const T x = a[i];
+        const int64_t x = a[i];
         a[i] = acc;
         acc += x;
     }
@@ -58,7 +60,7 @@ __device__ void block_exclusive_scan(T* a, int n, T* partial) {
 }
 
 // first index i in [0, n) with a[i] >= x (a non-decreasing), n if none
-__device__ __forceinline__ int lower_bound64(const int64_t* a, int n, int64_t x) {
+__device__ __noinline__ int lower_bound64(const int64_t* a, int n, int64_t x) {
     int lo = 0, hi = n;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
@@ -68,8 +70,10 @@ __device__ __forceinline__ int lower_bound64(const int64_t* a, int n, int64_t x)
 }
 
 // One CTA, everything in shared memory and in parallel:
-//   pre[b]   pages before request b (exclusive scan of ceil(T_b / 64));
-//   cuts[g]  share boundaries floor(total * g / G);
+//   pk[b]    (pages before request b) << 32 | (requests with tokens before b): one scan of
+//            (ceil(T_b / 64) << 32 | [T_b > 0]); the low field never carries into the high one;
+//   cut(g)   share boundary floor(total * g / G), and the first g whose cut is >= x in
+//            closed form, ceil(x * G / total);
 //   a cut that falls strictly inside a request, and is the first of its value, starts a new
 //   segment ("flagged"); every request with pages starts one;
 //   a request's segments are its start plus its flagged cuts; a group's first segment is
@@ -78,13 +82,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int H, WsLayout L, void* ws) {
     const int G = L.num_groups;
     extern __shared__ int64_t plan_sh[];
-    int64_t* pre = plan_sh;                                          // [B + 1]
-    int64_t* cuts = pre + (B + 1);                                   // [G + 1]
-    int64_t* part64 = cuts + (G + 1);                                // [kPlanThreads]
-    int32_t* nseg = reinterpret_cast<int32_t*>(part64 + kPlanThreads);  // [B + 1] -> segment base
-    int32_t* vcnt = nseg + (B + 1);                                  // [B + 1] valid requests before b
-    int32_t* flag = vcnt + (B + 1);                                  // [G + 2] -> flagged cuts before g
-    int32_t* part32 = flag + (G + 2);                                // [kPlanThreads]
+    int64_t* pk = plan_sh;             // [B + 1]
+    int64_t* flag = pk + (B + 1);      // [G + 2] -> flagged cuts before g
+    int64_t* nseg = flag + (G + 2);    // [B + 1] -> first segment of request b
+    int64_t* part = nseg + (B + 1);    // [16] scan scratch
     __shared__ int bad_first;
     PlanHeader* h = reinterpret_cast<PlanHeader*>(ws);
     int32_t* group_begin = ws_ptr<int32_t>(ws, L.off_group_begin);
@@ -99,68 +100,77 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     __syncthreads();
     for (int b = tid; b < B; b += kPlanThreads) {
         const int T = seq_lens[b];
-        pre[b] = T > 0 ? (T + kPage - 1) / kPage : 0;
-        vcnt[b] = T > 0 ? 1 : 0;
+        pk[b] = T > 0 ? ((int64_t)((T + kPage - 1) / kPage) << 32) | 1 : 0;
         if (T <= 0) atomicMin(&bad_first, b);
     }
     __syncthreads();
-    block_exclusive_scan(pre, B, part64);
-    block_exclusive_scan(vcnt, B, part32);
-    const int64_t total = pre[B];
-    for (int g = tid; g <= G; g += kPlanThreads) cuts[g] = total * (int64_t)g / G;
-    __syncthreads();
+    block_exclusive_scan(pk, B, part);
+    const int64_t total = pk[B] >> 32;
+    // first g in [0, G] with cut(g) >= x; G + 1 if none
+    auto first_cut_ge = [&](int64_t x) -> int {
+        if (x <= 0) return 0;
+        if (x > total) return G + 1;
+        return (int)((x * G + total - 1) / total);
+    };
     for (int g = tid; g <= G; g += kPlanThreads) {
-        int f = 0;
-        const int64_t cg = cuts[g];
-        if (g > 0 && g < G && cg > 0 && cg < total && cg != cuts[g - 1]) {
-            // a request start? the last request whose start is <= cg starts exactly at cg and
-            // has pages
-            const int bl = lower_bound64(pre, B + 1, cg + 1) - 1;
-            const bool is_start = bl < B && pre[bl] == cg && pre[bl + 1] > cg;
-            f = is_start ? 0 : 1;
+        int64_t f = 0;
+        if (g > 0 && g < G) {
+            const int64_t cg = total * g / G;
+            if (cg > 0 && cg < total && cg != total * (g - 1) / G) {
+                // a request start? the last request whose start is <= cg starts exactly at cg
+                // and has pages
+                const int bl = lower_bound64(pk, B + 1, (cg + 1) << 32) - 1;
+                const bool is_start = bl < B && (pk[bl] >> 32) == cg && (pk[bl + 1] >> 32) > cg;
+                f = is_start ? 0 : 1;
+            }
         }
         flag[g] = f;
     }
     __syncthreads();
-    block_exclusive_scan(flag, G + 1, part32);  // flag[g] = flagged cuts with index < g
+    block_exclusive_scan(flag, G + 1, part);  // flag[g] = flagged cuts with index < g
     for (int b = tid; b < B; b += kPlanThreads) {
-        const int64_t p0 = pre[b], p1 = pre[b + 1];
-        int n = 0;
+        const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
+        int64_t n = 0;
         if (p1 > p0) {
-            const int gl = lower_bound64(cuts, G + 1, p0 + 1);  // first cut > p0
-            const int gh = lower_bound64(cuts, G + 1, p1);      // first cut >= p1
+            const int gl = first_cut_ge(p0 + 1), gh = first_cut_ge(p1);
             n = 1 + (gh > gl ? flag[gh] - flag[gl] : 0);
         }
         nseg[b] = n;
     }
     __syncthreads();
-    block_exclusive_scan(nseg, B, part32);  // nseg[b] = first segment of request b
-    const int nseg_total = nseg[B];
+    block_exclusive_scan(nseg, B, part);  // nseg[b] = first segment of request b
+    const int nseg_total = (int)nseg[B];
+    // segment starts, in parallel: every request with pages starts its first segment at
+    // tile 0, every flagged cut starts the next segment of the request it falls in
     for (int b = tid; b < B; b += kPlanThreads) {
-        req_seg[b] = nseg[b];
-        const int64_t p0 = pre[b], p1 = pre[b + 1];
+        req_seg[b] = (int)nseg[b];
+        const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
         if (p1 <= p0) continue;
-        const int n = nseg[b + 1] - nseg[b];
-        const int gl = lower_bound64(cuts, G + 1, p0 + 1);
-        const int gh = lower_bound64(cuts, G + 1, p1);
-        int k = nseg[b];
-        int64_t start = p0;
-        for (int g = gl; g < gh; ++g) {
-            if (flag[g + 1] == flag[g]) continue;  // not a flagged cut
-            Segment sg;
-            sg.b = b;
-            sg.tile_begin = (int32_t)(start - p0);
-            sg.tile_end = (int32_t)(cuts[g] - p0);
-            sg.split = n > 1;
-            segs[k++] = sg;
-            start = cuts[g];
-        }
         Segment sg;
         sg.b = b;
-        sg.tile_begin = (int32_t)(start - p0);
-        sg.tile_end = (int32_t)(p1 - p0);
-        sg.split = n > 1;
-        segs[k] = sg;
+        sg.tile_begin = 0;
+        sg.tile_end = 0;  // set below
+        sg.split = nseg[b + 1] - nseg[b] > 1;
+        segs[nseg[b]] = sg;
+    }
+    for (int g = tid + 1; g < G; g += kPlanThreads) {
+        if (flag[g + 1] == flag[g]) continue;  // not a flagged cut
+        const int64_t cg = total * g / G;
+        const int b = lower_bound64(pk, B + 1, (cg + 1) << 32) - 1;  // the request cg falls strictly inside
+        const int64_t p0 = pk[b] >> 32;
+        Segment sg;
+        sg.b = b;
+        sg.tile_begin = (int32_t)(cg - p0);
+        sg.tile_end = 0;
+        sg.split = 1;
+        segs[nseg[b] + 1 + (flag[g] - flag[first_cut_ge(p0 + 1)])] = sg;
+    }
+    __syncthreads();
+    // each segment ends where the next one of its request starts, or at the request's end
+    for (int k = tid; k < nseg_total; k += kPlanThreads) {
+        const int b = __ldcg(&segs[k].b);
+        const bool last = k + 1 == nseg_total || __ldcg(&segs[k + 1].b) != b;
+        segs[k].tile_end = last ? (int32_t)((pk[b + 1] >> 32) - (pk[b] >> 32)) : __ldcg(&segs[k + 1].tile_begin);
     }
     for (int g = tid; g <= G; g += kPlanThreads) {
         int v;
@@ -169,11 +179,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         } else if (g == G) {
             v = nseg_total;
         } else {
-            // segment starts below cuts[g]: request starts below it plus flagged cuts below it
-            const int64_t x = cuts[g];
-            const int bx = lower_bound64(pre, B, x);           // requests 0..bx-1 start below x
-            const int gf = lower_bound64(cuts, G + 1, x);      // first cut of this value
-            v = vcnt[bx] + flag[gf];
+            // segment starts below cut(g): request starts below it plus flagged cuts below it
+            const int64_t x = total * g / G;
+            const int bx = lower_bound64(pk, B, x << 32);  // requests 0..bx-1 start below x
+            v = (int)(pk[bx] & 0xffffffff) + (int)flag[first_cut_ge(x)];
         }
         group_begin[g] = v;
     }
@@ -250,8 +259,7 @@ extern "C" mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, i
     WsLayout L = make_layout(B, s_q, H, num_groups_for(num_sms, num_row_blocks(s_q, H)));
     if (L.num_groups > kMaxGroups) return MLA_ERR_UNSUPPORTED;
     if ((int64_t)ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
-    const size_t smem = sizeof(int64_t) * ((size_t)B + 1 + (size_t)L.num_groups + 1 + kPlanThreads) +
-                        sizeof(int32_t) * (2 * ((size_t)B + 1) + (size_t)L.num_groups + 2 + kPlanThreads);
+    const size_t smem = sizeof(int64_t) * (2 * ((size_t)B + 1) + (size_t)L.num_groups + 2 + 16);
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
