@@ -126,8 +126,9 @@ mla_status mla_decode_scan(const void* q, const void* kv_pages, int kv_dtype, fl
  * The LSE-weighted combine of the split partials held in `workspace`: for every row of
  * a request that the plan split, lse = ln sum_j exp(lse_j) and
  * out = sum_j exp(lse_j - lse) * out_j (bf16); empty splits (lse_j = -inf) drop out.
- * Rows of unsplit requests are left untouched.  mla_decode calls it; it is exported so
- * that it can be run (and timed) on its own.
+ * Rows of unsplit requests are left untouched, and the rows of a request with
+ * seq_len <= 0 (which the plan gives no split) are written as NaN here, not by the scan.
+ * mla_decode calls it; it is exported so that it can be run (and timed) on its own.
  */
 mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, int s_q, int H,
                                 void* out, float* lse, void* stream);

@@ -37,9 +37,20 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __
     if (row0 >= M) return;
     const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
     const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
-    if (ns <= 1) return;  // written directly by the decode kernel
-    const int nqb = h->nqb;
     const int tid = threadIdx.x, r16 = tid & 15, cq = tid >> 4;
+    if (ns == 0) {
+        // a request without tokens (T_b <= 0) has no split: the planner set the status word,
+        // and its rows are written here as NaN
+        const int m = row0 + r16;
+        if (m < M) {
+            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
+                make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+            if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
+        }
+        return;
+    }
+    if (ns == 1) return;  // written directly by the decode kernel
+    const int nqb = h->nqb;
     // split j: partial tile at pbase + j * jstride (float4), lse2 of row r at lbase[j * lstride + r]
     const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
                           ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + (16 * c64 + cq) * 16 + r16;

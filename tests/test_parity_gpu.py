@@ -58,6 +58,29 @@ def test_edge_cases(kw, num_sms):
     _case("agent_spec", num_sms, **kw)
 
 
+def test_many_short_requests():
+    """More requests than the planner has threads: every planner loop runs several rounds."""
+    _case("agent_spec", 0, B=300, s_q=1, H=16, seq=("uniform", 1, 1500))
+
+
+def test_zero_length_request_is_reported_and_poisons_only_its_rows():
+    import torch
+    import mla_attention_decode_paged_b200 as mla
+    wl = W.make_workload("agent_spec", B=3, seq=("fixed", 700))
+    q, kv, bt, sl = pu.to_device(wl)
+    sl0 = torch.tensor([700, 0, 700], dtype=torch.int32, device="cuda")
+    ws = mla.alloc_workspace(3, wl.s_q, wl.H)
+    out = torch.zeros((3, wl.s_q, wl.H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((3, wl.s_q, wl.H), dtype=torch.float32, device="cuda")
+    mla.plan(sl0, wl.s_q, wl.H, ws)
+    mla.decode(q, kv, bt, sl0, wl.scale, True, ws, out, lse)
+    assert mla.device_status(ws) == 5
+    o = out.float().cpu().numpy()
+    assert np.all(np.isnan(o[1]))
+    ref_out, ref_lse = pu.run_oracle(wl, requests=[0, 2])
+    pu.check_close(o[[0, 2]], lse.cpu().numpy()[[0, 2]], ref_out, ref_lse, wl.kv_dtype, what="zero-length neighbour")
+
+
 def test_split_count_does_not_change_the_result_beyond_rounding():
     wl = W.make_workload("long_m256", B=2, seq=("fixed", 3000))
     a_out, a_lse = pu.run_gpu(wl, num_sms=4)      # one split per request (4 row blocks, 1 group)
@@ -94,7 +117,9 @@ def _read_plan(ws):
 
 
 @pytest.mark.parametrize("lens,s_q,H,num_sms", [([65536] * 4, 4, 16, 148), ([70000, 1, 64, 65, 30000], 2, 128, 148),
-                                                ([300] * 3, 8, 32, 8), ([5] * 7, 1, 16, 1)])
+                                                ([300] * 3, 8, 32, 8), ([5] * 7, 1, 16, 1),
+                                                (list(np.random.default_rng(1).integers(1, 3000, 600)), 1, 16, 148),
+                                                ([0, 100, 0, 5000], 1, 16, 148)])
 def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     import torch
     import mla_attention_decode_paged_b200 as mla

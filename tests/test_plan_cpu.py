@@ -9,7 +9,9 @@ from tests import plan_ref
 
 
 @pytest.mark.parametrize("lens,G", [([65536] * 4, 74), ([256], 74), ([65, 129], 74), ([100, 5000, 64, 1], 3),
-                                    (list(np.random.default_rng(0).integers(1, 70000, 32)), 37), ([64] * 10, 1)])
+                                    (list(np.random.default_rng(0).integers(1, 70000, 32)), 37), ([64] * 10, 1),
+                                    (list(np.random.default_rng(1).integers(1, 3000, 600)), 148),
+                                    (list(np.random.default_rng(2).integers(1, 200, 1000)), 1023)])
 def test_plan_covers_every_page_once_in_order_and_balances(lens, G):
     gb, rs, segs = plan_ref.plan(lens, G)
     tiles = [(t + 63) // 64 for t in lens]
