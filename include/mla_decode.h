@@ -134,6 +134,18 @@ mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, i
                                 void* out, float* lse, void* stream);
 
 /*
+ * Test and debugging aid for the device-side failure detection (no counterpart on the
+ * pages).  Every wait of the scan kernel on an mbarrier is bounded: after its limit (2 s)
+ * the CTA gives up, records MLA_ERR_DEVICE_TIMEOUT in the workspace status word and
+ * returns, so that a lost arrival never hangs the GPU.  This call runs that same wait
+ * code in one thread on a barrier that nothing arrives at, with a 20 ms limit; afterwards
+ * mla_get_device_status reports MLA_ERR_DEVICE_TIMEOUT and the context stays usable.
+ * `workspace` needs only the 96-byte status header (256-byte aligned); a plan stored in
+ * it is left intact.  Returns MLA_ERR_INVALID_ARG / MLA_ERR_WORKSPACE_TOO_SMALL / MLA_OK.
+ */
+mla_status mla_debug_wait_timeout(void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Reads and clears the device status word of `workspace` (host out: *code, one of
  * MLA_OK, MLA_ERR_DEVICE_OOB, MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_PLAN_MISMATCH).  This
  * call synchronises `stream`; it is meant for tests and debugging.

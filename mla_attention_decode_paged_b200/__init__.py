@@ -36,10 +36,11 @@ def workspace_bytes(B: int, s_q: int, H: int, num_sms: int = 0) -> int:
 
 
 def alloc_workspace(B: int, s_q: int, H: int, num_sms: int = 0, device=None):
-    """A uint8 CUDA tensor large enough (and 256-byte aligned) for plan + decode."""
+    """A zero-filled uint8 CUDA tensor large enough (and 256-byte aligned) for plan + decode;
+    zero-filled so that its status word starts clear."""
     import torch
     n = workspace_bytes(B, s_q, H, num_sms)
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def plan(seq_lens, s_q: int, H: int, workspace, num_sms: int = 0, stream=None):

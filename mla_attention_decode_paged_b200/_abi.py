@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.mla_split_kv_combine.restype = I
         L.mla_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.mla_get_device_status.restype = I
+        L.mla_debug_wait_timeout.argtypes = [P, SZ, P]
+        L.mla_debug_wait_timeout.restype = I
         L.mla_decode_version.argtypes = []
         L.mla_decode_version.restype = ctypes.c_char_p
         _lib = L
@@ -101,6 +103,11 @@ def mla_get_device_status(workspace_ptr, stream) -> tuple:
     code = ctypes.c_int(-1)
     rc = lib().mla_get_device_status(workspace_ptr, ctypes.byref(code), stream)
     return rc, code.value
+
+
+def mla_debug_wait_timeout(workspace_ptr, ws_bytes, stream) -> int:
+    """The scan kernel's bounded wait on a barrier nothing arrives at (20 ms limit)."""
+    return lib().mla_debug_wait_timeout(workspace_ptr, ws_bytes, stream)
 
 
 def mla_decode_version() -> str:

@@ -25,6 +25,9 @@ struct DecodeParams {
 
 mla_status launch_decode_simt(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
 mla_status launch_decode_sm100(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
+// One CTA that runs the scan kernel's bounded wait on a barrier nothing arrives at (20 ms
+// limit) and so sets the timeout status in the workspace header.
+mla_status launch_wait_timeout_probe(void* ws, cudaStream_t stream);
 // CTAs of the tensor-core scan kernel that the current device runs at once (one per
 // SM); the split plan is made for this many by default.
 int sm100_cta_slots();

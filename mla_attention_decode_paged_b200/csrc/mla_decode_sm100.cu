@@ -98,7 +98,8 @@ struct Ctx {
 
 // Bounded wait: gives up after kWaitLimitNs (sets the timeout status and the CTA abort
 // flag), or at once once the CTA is aborting.
-__device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
+template <uint64_t kLimitNs>
+__device__ __noinline__ bool wait_bar_for(const Ctx& c, uint32_t bar, uint32_t parity) {
     if (*c.abort) return false;
     uint64_t t0 = 0;
     for (uint32_t n = 1;; ++n) {
@@ -108,13 +109,16 @@ __device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parit
             const uint64_t now = ptx::globaltimer_ns();
             if (t0 == 0) {
                 t0 = now;
-            } else if (now - t0 > kWaitLimitNs) {
+            } else if (now - t0 > kLimitNs) {
                 *c.abort = 1;
                 set_status(c.h, kStatusTimeout, (int)blockIdx.x);
                 return false;
             }
         }
     }
+}
+__device__ __forceinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
+    return wait_bar_for<kWaitLimitNs>(c, bar, parity);
 }
 
 // Wait that ignores the abort flag, used only on the way out for work already in flight.
@@ -747,6 +751,29 @@ mla_status launch_typed(const DecodeParams& p, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, decode_sm100_kernel<KV>, a) != cudaSuccess) return MLA_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// The bounded wait of the scan kernel, on a barrier that nothing arrives at, with a 20 ms
+// limit: it gives up, sets the timeout status and returns.  A test of that mechanism
+// that needs no fault and no hang.
+__global__ void wait_timeout_probe_kernel(void* ws) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    abort_flag = 0;
+    const uint32_t b = ptx::smem_u32(&bar);
+    ptx::mbar_init(b, 1);
+    ptx::fence_mbar_init_cluster();
+    Ctx c;
+    c.bar0 = b;
+    c.abort = &abort_flag;
+    c.h = reinterpret_cast<PlanHeader*>(ws);
+    wait_bar_for<20000000ull>(c, b, 0);
+}
+
+mla_status launch_wait_timeout_probe(void* ws, cudaStream_t stream) {
+    wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(ws);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

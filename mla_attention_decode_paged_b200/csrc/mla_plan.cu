@@ -268,6 +268,12 @@ extern "C" mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, i
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+extern "C" mla_status mla_debug_wait_timeout(void* workspace, size_t ws_bytes, void* stream) {
+    if (!workspace || ((uintptr_t)workspace & 255) != 0) return MLA_ERR_INVALID_ARG;
+    if (ws_bytes < sizeof(PlanHeader)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    return launch_wait_timeout_probe(workspace, (cudaStream_t)stream);
+}
+
 extern "C" mla_status mla_get_device_status(void* workspace, int* code, void* stream) {
     if (!workspace || !code) return MLA_ERR_INVALID_ARG;
     int32_t h[2] = {0, 0};

@@ -95,3 +95,9 @@ def test_combine_rejects_bad_arguments():
 def test_status_query_rejects_null():
     rc, _ = _abi.mla_get_device_status(None, None)
     assert rc == _abi.MLA_ERR_INVALID_ARG
+
+
+def test_timeout_probe_rejects_bad_workspace_before_any_launch():
+    assert _abi.mla_debug_wait_timeout(None, 1 << 20, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_debug_wait_timeout(256 + 16, 1 << 20, None) == _abi.MLA_ERR_INVALID_ARG  # not 256-aligned
+    assert _abi.mla_debug_wait_timeout(256, 64, None) == _abi.MLA_ERR_WORKSPACE_TOO_SMALL

@@ -178,3 +178,21 @@ def test_full_size_workload_sampled_rows(name):
     got_lse = lse[reqs][:, :, heads]
     pu.check_close(got_out, got_lse, ref_out, ref_lse, wl.kv_dtype, what=name)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+
+
+def test_bounded_wait_gives_up_with_a_status_and_the_context_stays_usable():
+    """The scan kernel's mbarrier wait, run on a barrier that nothing arrives at, ends after
+    its limit with the timeout status instead of hanging; decoding works afterwards."""
+    import torch
+    import mla_attention_decode_paged_b200 as mla
+    from mla_attention_decode_paged_b200 import _abi
+    wl = W.make_workload("agent_spec", B=2, seq=("fixed", 900))
+    ws = mla.alloc_workspace(wl.B, wl.s_q, wl.H)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert mla.device_status(ws) == 0  # a fresh workspace starts with a clear status word
+    assert _abi.mla_debug_wait_timeout(ws.data_ptr(), ws.numel(), stream) == 0
+    assert mla.device_status(ws) == 6  # MLA_ERR_DEVICE_TIMEOUT
+    assert mla.device_status(ws) == 0
+    out, lse = pu.run_gpu(wl)
+    ref_out, ref_lse = pu.run_oracle(wl)
+    pu.check_close(out.reshape(ref_out.shape), lse, ref_out, ref_lse, wl.kv_dtype, what="after a timeout")
