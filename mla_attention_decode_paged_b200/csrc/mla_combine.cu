@@ -9,24 +9,29 @@
 // it drops out.  The kernel reads every partial once; it is bound by that read.
 #include <string.h>
 
-#include "mla_common.cuh"
+#include "mla_decode_params.cuh"
 
 namespace mla {
 
-constexpr int kCombineThreads = 256;  // 16 rows x 16 column quads
+constexpr int kTileThreads = 256;     // 16 rows x 16 column quads
 constexpr int kWChunk = 64;           // splits whose weights are in shared memory at once
-constexpr int kPre = 8;               // partials loaded before the weights are known
+constexpr int kPre = 6;               // partials per thread loaded before the weights are known
 
-// grid (B, 4 nqb, 8): one CTA per (request, 16-row group, 64 columns).  Thread t owns row
-// t % 16 and column quad t / 16 of the tile; in the workspace's quad-interleaved partial
-// layout the CTA's tile of one split is 4 KB contiguous, read by the 256 threads with
-// one 16-byte load each.  The first kPre partials are loaded before the weights are
-// computed, so their latency overlaps that computation.
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __restrict__ ws, int B, int s_q, int H,
-                                                                  __nv_bfloat16* __restrict__ out,
-                                                                  float* __restrict__ lse) {
+// grid (B, 4 nqb, 8): one CTA per (request, 16-row group, 64 columns).  Within a group of
+// 256 threads, thread t owns row t % 16 and column quad t / 16 of the tile; in the
+// workspace's quad-interleaved partial layout the CTA's tile of one split is 4 KB
+// contiguous, read by the 256 threads with one 16-byte load each.  kSplitGroups groups
+// take the splits j = group, group + kSplitGroups, ... so that kSplitGroups x kPre
+// partials are in flight before the weights are known; the group sums meet in shared
+// memory at the end.  Four groups when requests have many splits (few long requests),
+// one when they have few (then more, smaller CTAs share an SM).
+template <int kSplitGroups>
+__global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups) combine_kernel(
+    const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    constexpr int kCombineThreads = kTileThreads * kSplitGroups;
     __shared__ float wsh[kWChunk][16];
     __shared__ float Lsh[16], Msh[16];
+    __shared__ float4 part[kSplitGroups > 1 ? kSplitGroups - 1 : 1][kTileThreads];
     const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
     // launched as a programmatic dependent of the scan: nothing is read before it completes
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -37,12 +42,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __
     if (row0 >= M) return;
     const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
     const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
-    const int tid = threadIdx.x, r16 = tid & 15, cq = tid >> 4;
+    const int tid = threadIdx.x, t = tid & (kTileThreads - 1), grp = tid / kTileThreads;
+    const int r16 = t & 15, cq = t >> 4;
     if (ns == 0) {
         // a request without tokens (T_b <= 0) has no split: the planner set the status word,
         // and its rows are written here as NaN
         const int m = row0 + r16;
-        if (m < M) {
+        if (grp == 0 && m < M) {
             *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
                 make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
             if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
@@ -60,10 +66,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __
 
     float4 v[kPre];
 #pragma unroll
-    for (int u = 0; u < kPre; ++u) v[u] = u < ns ? pbase[u * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kPre; ++u) {
+        const int j = grp + kSplitGroups * u;
+        v[u] = j < ns ? pbase[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 
-    // L = log2 sum_j 2^lse2_j per row: warp w takes rows 2w and 2w + 1 (one per half-warp)
-    {
+    // L = log2 sum_j 2^lse2_j per row: warp w < 8 takes rows 2w and 2w + 1 (one per half-warp)
+    if (tid < kTileThreads) {
         const int lane = tid & 31, r = 2 * (tid >> 5) + (lane >> 4), k = lane & 15;
         float mx = -INFINITY;
         for (int j = k; j < ns; j += 16) mx = fmaxf(mx, lbase[j * lstride + r]);
@@ -89,31 +98,42 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __
             wsh[jj][r] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - Lsh[r]);  // an empty split drops out
         }
         __syncthreads();
-        int jj = 0;
+        int jj = grp;  // this group's splits within the chunk: grp, grp + 4, ...
         if (j0 == 0) {
 #pragma unroll
             for (int u = 0; u < kPre; ++u) {
-                const float w = u < nj ? wsh[u][r16] : 0.f;
+                const int j = grp + kSplitGroups * u;
+                const float w = j < nj ? wsh[j][r16] : 0.f;
                 acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
             }
-            jj = kPre;
+            jj = grp + kSplitGroups * kPre;
         }
-        for (; jj + 3 < nj; jj += 4) {
-            float4 x[4];
+        for (; jj + kSplitGroups < nj; jj += 2 * kSplitGroups) {
+            float4 x[2];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) x[u] = pbase[(j0 + jj + u) * jstride];
+            for (int u = 0; u < 2; ++u) x[u] = pbase[(j0 + jj + kSplitGroups * u) * jstride];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float w = wsh[jj + u][r16];
+            for (int u = 0; u < 2; ++u) {
+                const float w = wsh[jj + kSplitGroups * u][r16];
                 acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
             }
         }
-        for (; jj < nj; ++jj) {
+        for (; jj < nj; jj += kSplitGroups) {
             const float4 x = pbase[(j0 + jj) * jstride];
             const float w = wsh[jj][r16];
             acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
         }
         __syncthreads();
+    }
+    if (kSplitGroups > 1) {
+        if (grp > 0) part[grp - 1][t] = acc;
+        __syncthreads();
+        if (grp > 0) return;
+#pragma unroll
+        for (int k = 0; k < kSplitGroups - 1; ++k) {
+            const float4 x = part[k][t];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
     }
     const int m = row0 + r16;
     if (m < M) {
@@ -128,19 +148,25 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const void* __
 }
 
 mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream) {
+    // a performance choice only (either kernel is correct for any plan): requests average
+    // (B + G) / B splits under the default plan
+    const int sms = effective_sms();
+    const int G = num_groups_for(sms > 0 ? sms : 1, num_row_blocks(s_q, H));
+    const bool many_splits = (int64_t)B + G >= 8 * (int64_t)B;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(B, 4 * num_row_blocks(s_q, H), kDv / 64);
-    cfg.blockDim = dim3(kCombineThreads);
+    cfg.blockDim = dim3(kTileThreads * (many_splits ? 4 : 1));
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, combine_kernel, ws, B, s_q, H, reinterpret_cast<__nv_bfloat16*>(out), lse) !=
-        cudaSuccess)
-        return MLA_ERR_CUDA;
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+    const cudaError_t e = many_splits ? cudaLaunchKernelEx(&cfg, combine_kernel<4>, ws, B, s_q, H, o, lse)
+                                      : cudaLaunchKernelEx(&cfg, combine_kernel<1>, ws, B, s_q, H, o, lse);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -140,16 +140,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     __syncthreads();
     block_exclusive_scan(nseg, B, part);  // nseg[b] = first segment of request b
     const int nseg_total = (int)nseg[B];
-    // segment starts, in parallel: every request with pages starts its first segment at
-    // tile 0, every flagged cut starts the next segment of the request it falls in
+    // segments, in parallel: every request with pages starts its first segment at tile 0,
+    // every flagged cut starts the next segment of the request it falls in; a segment ends
+    // at the next flagged cut inside its request (found by a search of the scanned flags:
+    // cut g is flagged iff flag[g + 1] > flag[g]) or at the request's end
     for (int b = tid; b < B; b += kPlanThreads) {
         req_seg[b] = (int)nseg[b];
         const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
         if (p1 <= p0) continue;
+        const int gl = first_cut_ge(p0 + 1), gh = first_cut_ge(p1);
+        const int g1 = lower_bound64(flag, G + 2, flag[gl] + 1) - 1;  // first flagged cut >= gl
         Segment sg;
         sg.b = b;
         sg.tile_begin = 0;
-        sg.tile_end = 0;  // set below
+        sg.tile_end = (int32_t)((g1 < gh ? total * g1 / G : p1) - p0);
         sg.split = nseg[b + 1] - nseg[b] > 1;
         segs[nseg[b]] = sg;
     }
@@ -157,20 +161,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         if (flag[g + 1] == flag[g]) continue;  // not a flagged cut
         const int64_t cg = total * g / G;
         const int b = lower_bound64(pk, B + 1, (cg + 1) << 32) - 1;  // the request cg falls strictly inside
-        const int64_t p0 = pk[b] >> 32;
+        const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
+        const int gh = first_cut_ge(p1);
+        const int g2 = lower_bound64(flag, G + 2, flag[g + 1] + 1) - 1;  // next flagged cut after g
         Segment sg;
         sg.b = b;
         sg.tile_begin = (int32_t)(cg - p0);
-        sg.tile_end = 0;
+        sg.tile_end = (int32_t)((g2 < gh ? total * g2 / G : p1) - p0);
         sg.split = 1;
         segs[nseg[b] + 1 + (flag[g] - flag[first_cut_ge(p0 + 1)])] = sg;
-    }
-    __syncthreads();
-    // each segment ends where the next one of its request starts, or at the request's end
-    for (int k = tid; k < nseg_total; k += kPlanThreads) {
-        const int b = __ldcg(&segs[k].b);
-        const bool last = k + 1 == nseg_total || __ldcg(&segs[k + 1].b) != b;
-        segs[k].tile_end = last ? (int32_t)((pk[b + 1] >> 32) - (pk[b] >> 32)) : __ldcg(&segs[k + 1].tile_begin);
     }
     for (int g = tid; g <= G; g += kPlanThreads) {
         int v;
