@@ -43,7 +43,8 @@ def build(force: bool = False) -> str:
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"]
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off", "-o", tmp, _SRC,
+               "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -65,6 +66,14 @@ def _load():
             lib.oracle_e4m3_to_double.restype = f64
             lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
             lib.oracle_bf16_to_double.restype = f64
+            lib.oracle_rope_table.argtypes = [i32, f64, P]
+            lib.oracle_rope_table.restype = None
+            lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+            lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+            lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+            lib.oracle_kv_append.argtypes = [P, P, P, i32, P, i32, ctypes.c_float, P, i32, P, i32, i32, i64, i32]
+            lib.oracle_kv_append.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -124,3 +133,43 @@ def e4m3_to_double(byte: int) -> float:
 
 def bf16_to_double(bits: int) -> float:
     return _load().oracle_bf16_to_double(int(bits) & 0xFFFF)
+
+
+def rope_table(max_pos: int, base: float = 10000.0):
+    """float32 [max_pos, 64]: cos(pos * base^(-2j/64)) for j < 32, then the sines."""
+    t = np.zeros((max_pos, 64), dtype=np.float32)
+    _load().oracle_rope_table(int(max_pos), float(base), _ptr(t))
+    return t
+
+
+def f32_to_bf16(x: float) -> int:
+    return int(_load().oracle_f32_to_bf16(float(x)))
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(_load().oracle_f32_to_e4m3(float(x)))
+
+
+def kv_append(ckv_bits, kpe_bits, cos_sin, kv, kv_dtype, kv_scale, block_table, seq_lens, page=PAGE):
+    """Reference of the paged KV append, in place on a copy of ``kv`` (returned).
+
+    ckv_bits uint16 [B, s_q, 512] and kpe_bits uint16 [B, s_q, 64] (bf16 bit patterns);
+    cos_sin float32 [max_pos, 64]; kv uint16 / uint8 [P, page, 576].  Raises on a length
+    or page id out of range.
+    """
+    lib = _load()
+    ckv_bits = np.ascontiguousarray(ckv_bits, dtype=np.uint16)
+    kpe_bits = np.ascontiguousarray(kpe_bits, dtype=np.uint16)
+    B, s_q, d = ckv_bits.shape
+    assert d == DV and kpe_bits.shape == (B, s_q, 64)
+    cs = np.ascontiguousarray(cos_sin, dtype=np.float32)
+    out = np.array(kv, copy=True, order="C")
+    assert out.dtype == (np.uint16 if kv_dtype == KV_BF16 else np.uint8)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    rc = lib.oracle_kv_append(_ptr(ckv_bits), _ptr(kpe_bits), _ptr(cs), int(cs.shape[0]), _ptr(out), int(kv_dtype),
+                              float(kv_scale), _ptr(bt), int(bt.shape[1]), _ptr(sl), B, s_q, int(out.shape[0]),
+                              int(page))
+    if rc != 0:
+        raise ValueError("oracle rejected a length or page id")
+    return out

@@ -239,3 +239,104 @@ void oracle_combine(const double* outs, const double* lses, int n, int64_t rows,
         lse[r] = L;
     }
 }
+
+/* ------------------------------------------------------------------ paged KV append
+ *
+ * The write side of the same cache.  The s_q new latent rows of request b (the draft
+ * tokens under verification) take the positions
+ *     pos_i = T_b - s_q + i          (seq_lens counts them, as in the decode above)
+ * and row pos of request b is pool[ block_table[b][pos / page] ][ pos % page ]
+ * [llm-atlas "Inference systems", 07 PagedAttention].
+ *   columns 0..511   = c_kv of the new token, stored as given (an e4m3 cache stores its
+ *                      quantised value);
+ *   columns 512..575 = the decoupled rope key rotated by its position
+ *                      [llm-atlas "Inference systems", 22 DeepSeek V2->V3].
+ * Rotation (reading: adjacent pairs, as in the RoFormer formulation): for j < 32
+ *     (x[2j], x[2j+1]) -> (x[2j] c_j - x[2j+1] s_j,  x[2j] s_j + x[2j+1] c_j),
+ *     c_j = cos(pos * theta_j), s_j = sin(pos * theta_j), theta_j = base^(-2j/64).
+ * The caller passes c and s as a float table [max_pos][64] (the 32 cosines, then the 32
+ * sines), the precomputed rope cache serving engines carry; oracle_rope_table builds it
+ * from the formula in float64 and rounds each entry to float.
+ * The stored value is a rounding decision, so it is taken in one stated precision:
+ * every product and sum in IEEE binary32, round to nearest, no fused multiply-add; then
+ * bf16 (nearest, ties to even) or, for an e4m3 cache, e4m3 of (value / kv_scale) with
+ * the division in binary32 (nearest, ties to the even code, saturating at +-448, NaN
+ * kept).
+ */
+
+void oracle_rope_table(int max_pos, double base, float* table) {
+    for (int pos = 0; pos < max_pos; ++pos)
+        for (int j = 0; j < 32; ++j) {
+            const double theta = pow(base, -2.0 * j / 64.0);
+            table[(int64_t)pos * 64 + j] = (float)cos(pos * theta);
+            table[(int64_t)pos * 64 + 32 + j] = (float)sin(pos * theta);
+        }
+}
+
+/* binary32 -> bfloat16 bits, round to nearest, ties to even; NaN stays NaN. */
+uint16_t oracle_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    const uint32_t lsb = (u >> 16) & 1u;
+    return (uint16_t)((u + 0x7FFFu + lsb) >> 16);
+}
+
+/* binary32 -> e4m3 byte: the nearest finite e4m3 value (ties to the even code, i.e. the
+ * one whose mantissa's last bit is 0), magnitudes past 448 saturate to 448, NaN -> NaN.
+ * Written as a search over the 127 non-negative finite codes. */
+uint8_t oracle_f32_to_e4m3(float f) {
+    if (f != f) return 0x7F;
+    const uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    const double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;
+    int best = 0;
+    double best_err = INFINITY;
+    for (int code = 0; code <= 0x7E; ++code) {
+        const double err = fabs(oracle_e4m3_to_double((uint8_t)code) - a);
+        if (err < best_err || (err == best_err && (code & 1) == 0)) {
+            best = code;
+            best_err = err;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* Returns 0, or -1 if some request was skipped (length or page id out of range). */
+int oracle_kv_append(const uint16_t* ckv, const uint16_t* kpe, const float* cos_sin, int max_pos, void* pool,
+                     int kv_dtype, float kv_scale, const int32_t* block_table, int max_pages,
+                     const int32_t* seq_lens, int B, int s_q, int64_t num_pages, int page) {
+    int rc = 0;
+    for (int b = 0; b < B; ++b) {
+        const int T = seq_lens[b];
+        if (T < s_q || T > (int64_t)max_pages * page) { rc = -1; continue; }
+        for (int i = 0; i < s_q; ++i) {
+            const int pos = T - s_q + i;
+            const int32_t pg = block_table[(int64_t)b * max_pages + pos / page];
+            if (pg < 0 || pg >= num_pages || pos >= max_pos) { rc = -1; continue; }
+            const int64_t row = (int64_t)pg * page + pos % page;
+            const uint16_t* src = ckv + ((int64_t)b * s_q + i) * ORACLE_DV;
+            const uint16_t* rk = kpe + ((int64_t)b * s_q + i) * 64;
+            const float* cs = cos_sin + (int64_t)pos * 64;
+            float vals[ORACLE_DQK];
+            for (int d = 0; d < ORACLE_DV; ++d) vals[d] = (float)bf16_bits_to_double(src[d]);
+            for (int j = 0; j < 32; ++j) {
+                const float x0 = (float)bf16_bits_to_double(rk[2 * j]);
+                const float x1 = (float)bf16_bits_to_double(rk[2 * j + 1]);
+                const float c = cs[j], s = cs[32 + j];
+                const float p00 = x0 * c, p11 = x1 * s, p01 = x0 * s, p10 = x1 * c;
+                vals[ORACLE_DV + 2 * j] = p00 - p11;
+                vals[ORACLE_DV + 2 * j + 1] = p01 + p10;
+            }
+            if (kv_dtype == ORACLE_KV_BF16) {
+                uint16_t* dst = (uint16_t*)pool + row * ORACLE_DQK;
+                for (int d = 0; d < ORACLE_DV; ++d) dst[d] = src[d];
+                for (int d = ORACLE_DV; d < ORACLE_DQK; ++d) dst[d] = oracle_f32_to_bf16(vals[d]);
+            } else {
+                uint8_t* dst = (uint8_t*)pool + row * ORACLE_DQK;
+                for (int d = 0; d < ORACLE_DQK; ++d) dst[d] = oracle_f32_to_e4m3(vals[d] / kv_scale);
+            }
+        }
+    }
+    return rc;
+}
