@@ -361,6 +361,29 @@ def run_ours(args):
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
+    # the write side of the same cache: append the s_q draft rows of each request (rope on
+    # the 64-wide key), timed on its own after everything above (it rewrites those rows)
+    ckv_new = torch.randn((wl.B, wl.s_q, W.DV), device=dev).to(torch.bfloat16)
+    kpe_new = torch.randn((wl.B, wl.s_q, 64), device=dev).to(torch.bfloat16)
+    max_pos = int(wl.seq_lens.max()) + 1
+    ang = torch.arange(max_pos, device=dev, dtype=torch.float64)[:, None] * \
+        (10000.0 ** (-torch.arange(32, device=dev, dtype=torch.float64) / 32.0))[None, :]
+    cos_sin = torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).float().contiguous()
+    app_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for k in range(args.warmup):
+        mla.kv_append(ckv_new, kpe_new, cos_sin, kv, bt, sl, kv_scale=wl.kv_scale, stream=stream)
+    for k in range(args.steps):
+        flush_l2(k)
+        app_ev[k][0].record(stream)
+        mla.kv_append(ckv_new, kpe_new, cos_sin, kv, bt, sl, kv_scale=wl.kv_scale, stream=stream)
+        app_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    app_us = statistics.median(e[0].elapsed_time(e[1]) for e in app_ev) * 1e3
+    elem = 2 if wl.kv_dtype == W.KV_BF16 else 1
+    app_bytes = wl.B * wl.s_q * (W.DV * 2 + 64 * 2 + 64 * 4 + W.DQK * elem)
+    kv_append_line = {"us_per_call": app_us, "bytes_per_call": app_bytes, "GB/s": app_bytes / (app_us * 1e-6) / 1e9,
+                      "rows": wl.B * wl.s_q, "note": "launch-bound at decode sizes; L2 flushed before each call"}
+
     kvb = wl.kv_bytes()
     flops = wl.flops()
     value = kvb * world * args.steps / (tot_ms * 1e-3) / 1e9
@@ -406,6 +429,7 @@ def run_ours(args):
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "us_per_call": float(e2e_tot[0]) / args.steps * 1e3,
                     "note": "q, block_table, seq_lens in and out, lse out per step; the paged cache stays resident"},
+            "kv_append": kv_append_line,
             "gpu_launches": 3 * args.steps,
             "gpu_launches_per_kernel_pass": 3 * args.steps,
             "gpu_launches_graph_pass": 3 * args.steps,

@@ -134,6 +134,34 @@ mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, i
                                 void* out, float* lse, void* stream);
 
 /*
+ * Paged KV append: the write side of the same cache (the step after the decode in the
+ * scope table).  The s_q new latent rows of request b -- the draft tokens the decode
+ * verifies, counted in seq_lens -- are stored at positions T_b - s_q + i, row
+ * pool[block_table[b][pos / 64]][pos % 64] (paging: llm-atlas "Inference systems", 07
+ * PagedAttention), with the 64-wide decoupled rope key rotated by its position (22
+ * DeepSeek V2->V3):
+ *   ckv_new       bf16 [B, s_q, 512], 16-byte aligned: the latent c_kv rows, stored as
+ *                 given (an e4m3 cache stores e4m3(value / kv_scale));
+ *   kpe_new       bf16 [B, s_q, 64]: the rope key before rotation; pairs (2j, 2j+1) are
+ *                 rotated: (x0 c_j - x1 s_j, x0 s_j + x1 c_j);
+ *   rope_cos_sin  float [max_pos, 64]: for each position the 32 cosines, then the 32
+ *                 sines (the caller's precomputed rope cache); positions >= max_pos are
+ *                 an error;
+ *   kv_pages, kv_dtype, kv_scale, block_table, max_pages_per_req, num_pages: the cache,
+ *                 as for mla_decode (kv_scale > 0 for e4m3, ignored for bf16);
+ *   status        optional device int32: set to MLA_ERR_DEVICE_OOB (if it was 0) for a
+ *                 request whose length (T_b < s_q or > max_pages * 64), position or page
+ *                 id is out of range; its rows are not written.  May be NULL.
+ * Arithmetic: binary32 products and sums each rounded (no fused multiply-add), then
+ * bf16 round-to-nearest-even, or e4m3 of a rounded binary32 division, round-to-nearest-
+ * even, saturating at +-448.  Argument errors return before any launch.
+ */
+mla_status mla_kv_append(const void* ckv_new, const void* kpe_new, const float* rope_cos_sin, int max_pos,
+                         void* kv_pages, int kv_dtype, float kv_scale, const int32_t* block_table,
+                         int max_pages_per_req, const int32_t* seq_lens, int B, int s_q, int64_t num_pages,
+                         int32_t* status, void* stream);
+
+/*
  * Test and debugging aid for the device-side failure detection (no counterpart on the
  * pages).  Every wait of the scan kernel on an mbarrier is bounded: after its limit (2 s)
  * the CTA gives up, records MLA_ERR_DEVICE_TIMEOUT in the workspace status word and

@@ -9,7 +9,7 @@ from __future__ import annotations
 
 from . import _abi
 from ._abi import (MLA_KV_BF16, MLA_KV_E4M3, MlaError, mla_decode_plan, mla_decode_version,
-                   mla_decode_workspace_size, mla_get_device_status, mla_split_kv_combine)
+                   mla_decode_workspace_size, mla_get_device_status, mla_kv_append, mla_split_kv_combine)
 
 PAGE = 64
 DQK = 576
@@ -89,3 +89,19 @@ def device_status(workspace, stream=None) -> int:
     rc, code = mla_get_device_status(workspace.data_ptr(), _stream_ptr(stream))
     _check(rc, "mla_get_device_status")
     return code
+
+
+def kv_append(ckv_new, kpe_new, rope_cos_sin, kv_pages, block_table, seq_lens, kv_scale: float = 1.0,
+              status=None, stream=None):
+    """Write the s_q new latent rows of each request into the paged cache (the draft
+    tokens, positions T_b - s_q + i), rotating their rope key (see mla_kv_append in
+    include/mla_decode.h).  ckv_new bf16 [B, s_q, 512], kpe_new bf16 [B, s_q, 64],
+    rope_cos_sin float32 [max_pos, 64]; kv_pages bf16 or float8_e4m3fn / uint8
+    [P, 64, 576]; status: optional int32 CUDA tensor of one element."""
+    import torch
+    B, s_q, _ = ckv_new.shape
+    kv_dtype = MLA_KV_BF16 if kv_pages.dtype == torch.bfloat16 else MLA_KV_E4M3
+    _check(mla_kv_append(ckv_new.data_ptr(), kpe_new.data_ptr(), rope_cos_sin.data_ptr(), rope_cos_sin.shape[0],
+                         kv_pages.data_ptr(), kv_dtype, float(kv_scale), block_table.data_ptr(), block_table.shape[1],
+                         seq_lens.data_ptr(), B, s_q, kv_pages.shape[0],
+                         None if status is None else status.data_ptr(), _stream_ptr(stream)), "mla_kv_append")

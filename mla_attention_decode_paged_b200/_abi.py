@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.mla_split_kv_combine.restype = I
         L.mla_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.mla_get_device_status.restype = I
+        L.mla_kv_append.argtypes = [P, P, P, I, P, I, F, P, I, P, I, I, I64, P, P]
+        L.mla_kv_append.restype = I
         L.mla_debug_wait_timeout.argtypes = [P, SZ, P]
         L.mla_debug_wait_timeout.restype = I
         L.mla_decode_version.argtypes = []
@@ -103,6 +105,12 @@ def mla_get_device_status(workspace_ptr, stream) -> tuple:
     code = ctypes.c_int(-1)
     rc = lib().mla_get_device_status(workspace_ptr, ctypes.byref(code), stream)
     return rc, code.value
+
+
+def mla_kv_append(ckv_ptr, kpe_ptr, cos_sin_ptr, max_pos, kv_ptr, kv_dtype, kv_scale, block_table_ptr,
+                  max_pages_per_req, seq_lens_ptr, B, s_q, num_pages, status_ptr, stream) -> int:
+    return lib().mla_kv_append(ckv_ptr, kpe_ptr, cos_sin_ptr, max_pos, kv_ptr, kv_dtype, kv_scale, block_table_ptr,
+                               max_pages_per_req, seq_lens_ptr, B, s_q, num_pages, status_ptr, stream)
 
 
 def mla_debug_wait_timeout(workspace_ptr, ws_bytes, stream) -> int:

@@ -101,3 +101,20 @@ def test_timeout_probe_rejects_bad_workspace_before_any_launch():
     assert _abi.mla_debug_wait_timeout(None, 1 << 20, None) == _abi.MLA_ERR_INVALID_ARG
     assert _abi.mla_debug_wait_timeout(256 + 16, 1 << 20, None) == _abi.MLA_ERR_INVALID_ARG  # not 256-aligned
     assert _abi.mla_debug_wait_timeout(256, 64, None) == _abi.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_kv_append_rejects_bad_arguments_before_any_launch():
+    ok = dict(ckv=256, kpe=256, cs=256, max_pos=100, kv=256, dt=0, scale=1.0, bt=256, mp=4, sl=256, B=2, s_q=4,
+              P=10, status=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return _abi.mla_kv_append(a["ckv"], a["kpe"], a["cs"], a["max_pos"], a["kv"], a["dt"], a["scale"], a["bt"],
+                                  a["mp"], a["sl"], a["B"], a["s_q"], a["P"], a["status"], None)
+    assert call(ckv=None) == _abi.MLA_ERR_INVALID_ARG
+    assert call(B=0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(max_pos=0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(dt=7) == _abi.MLA_ERR_INVALID_ARG
+    assert call(dt=1, scale=0.0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(ckv=256 + 8) == _abi.MLA_ERR_INVALID_ARG  # latent rows need 16-byte alignment
+    assert call(status=256 + 2) == _abi.MLA_ERR_INVALID_ARG
