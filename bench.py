@@ -191,6 +191,22 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(values, world, device):
+    """Per-rank totals reduced with MAX over the ranks: the slowest rank sets the job's
+    time.  Every rank calls it at the same points, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_gbs(bytes_per_rank_step, world, steps, total_ms):
+    """Whole-job throughput: every rank's bytes over the slowest rank's device time."""
+    return bytes_per_rank_step * world * steps / (total_ms * 1e-3) / 1e9
+
+
 def soak(step, flush_l2, dev, seconds):
     import torch
     t0 = time.perf_counter()
@@ -288,10 +304,7 @@ def run_ours(args):
     plan_ms = [e[0].elapsed_time(e[1]) for e in evs_split]
     scan_ms = [e[1].elapsed_time(e[2]) for e in evs_split]
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs_split]
-    tot = torch.tensor([sum(step_ms), sum(scan_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    tot_ms, tot_scan_ms = float(tot[0]), float(tot[1])
+    tot_ms, tot_scan_ms = max_over_ranks([sum(step_ms), sum(scan_ms)], world, dev)
 
     # the same step replayed from a CUDA graph (captured once; launch overhead removed)
     graph = None
@@ -316,11 +329,9 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         assert mla.device_status(ws, stream=stream) == 0
         gms = sorted(e[0].elapsed_time(e[1]) for e in gev)
-        gt = torch.tensor([sum(gms)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(gt, op=dist.ReduceOp.MAX)
-        graph = {"us_per_call": float(gt[0]) / args.steps * 1e3, "median_us": statistics.median(gms) * 1e3,
-                 "value": wl.kv_bytes() * world * args.steps / (float(gt[0]) * 1e-3) / 1e9, "unit": "GB/s"}
+        (g_ms,) = max_over_ranks([sum(gms)], world, dev)
+        graph = {"us_per_call": g_ms / args.steps * 1e3, "median_us": statistics.median(gms) * 1e3,
+                 "value": job_gbs(wl.kv_bytes(), world, args.steps, g_ms), "unit": "GB/s"}
         del g
     except Exception as e:  # reported, never fatal
         graph = {"error": f"{type(e).__name__}: {e}"[:200]}
@@ -355,9 +366,7 @@ def run_ours(args):
         flush_l2(k)
         e2e_step(e2e_ev[k])
     torch.cuda.synchronize(dev)
-    e2e_tot = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in e2e_ev)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_tot, op=dist.ReduceOp.MAX)
+    (e2e_ms,) = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in e2e_ev)], world, dev)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
@@ -386,8 +395,8 @@ def run_ours(args):
 
     kvb = wl.kv_bytes()
     flops = wl.flops()
-    value = kvb * world * args.steps / (tot_ms * 1e-3) / 1e9
-    e2e_value = kvb * world * args.steps / (float(e2e_tot[0]) * 1e-3) / 1e9
+    value = job_gbs(kvb, world, args.steps, tot_ms)
+    e2e_value = job_gbs(kvb, world, args.steps, e2e_ms)
     peaks, peak_src = load_peaks()
     scan_avg_s = tot_scan_ms * 1e-3 / args.steps
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -427,7 +436,7 @@ def run_ours(args):
                                     float(np.percentile(step_ms, 90)) * 1e3],
             "graph": graph,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "us_per_call": float(e2e_tot[0]) / args.steps * 1e3,
+                    "us_per_call": e2e_ms / args.steps * 1e3,
                     "note": "q, block_table, seq_lens in and out, lse out per step; the paged cache stays resident"},
             "kv_append": kv_append_line,
             "gpu_launches": 3 * args.steps,
