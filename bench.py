@@ -393,6 +393,37 @@ def run_ours(args):
     kv_append_line = {"us_per_call": app_us, "bytes_per_call": app_bytes, "GB/s": app_bytes / (app_us * 1e-6) / 1e9,
                       "rows": wl.B * wl.s_q, "note": "launch-bound at decode sizes; L2 flushed before each call"}
 
+    # the projections on either side of the latent attention, random weights (no model)
+    q_nope = torch.randn((wl.B, wl.s_q, wl.H, 128), device=dev).to(torch.bfloat16)
+    q_rope = torch.randn((wl.B, wl.s_q, wl.H, 64), device=dev).to(torch.bfloat16)
+    w_uk = (torch.randn((wl.H, W.DV, 128), device=dev) / 128 ** 0.5).to(torch.bfloat16)
+    w_uv = (torch.randn((wl.H, W.DV, 128), device=dev) / W.DV ** 0.5).to(torch.bfloat16)
+    q_abs = torch.empty((wl.B, wl.s_q, wl.H, W.DQK), dtype=torch.bfloat16, device=dev)
+    y_proj = torch.empty((wl.B, wl.s_q, wl.H, 128), dtype=torch.bfloat16, device=dev)
+
+    def time_op(fn):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for _ in range(args.warmup):
+            fn()
+        for k in range(args.steps):
+            flush_l2(k)
+            evs[k][0].record(stream)
+            fn()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.median(e[0].elapsed_time(e[1]) for e in evs) * 1e3
+
+    rows = wl.B * wl.s_q * wl.H
+    wbytes = wl.H * W.DV * 128 * 2
+    ab_us = time_op(lambda: mla.absorb_q(q_nope, q_rope, w_uk, q_abs, stream=stream))
+    pj_us = time_op(lambda: mla.project_out(out, w_uv, y_proj, stream=stream))
+    ab_bytes = wbytes + rows * (128 + 64 + W.DQK) * 2
+    pj_bytes = wbytes + rows * (W.DV + 128) * 2
+    absorb_line = {"absorb_q_us": ab_us, "absorb_q_GB/s": ab_bytes / (ab_us * 1e-6) / 1e9,
+                   "project_out_us": pj_us, "project_out_GB/s": pj_bytes / (pj_us * 1e-6) / 1e9,
+                   "weight_bytes_each": wbytes, "note": "per-head W_UK / W_UV [H, 512, 128] bf16, L2 flushed before "
+                                                       "each call; bound by the weights' bytes and launch latency"}
+
     kvb = wl.kv_bytes()
     flops = wl.flops()
     value = job_gbs(kvb, world, args.steps, tot_ms)
@@ -439,6 +470,7 @@ def run_ours(args):
                     "us_per_call": e2e_ms / args.steps * 1e3,
                     "note": "q, block_table, seq_lens in and out, lse out per step; the paged cache stays resident"},
             "kv_append": kv_append_line,
+            "absorb_project": absorb_line,
             "gpu_launches": 3 * args.steps,
             "gpu_launches_per_kernel_pass": 3 * args.steps,
             "gpu_launches_graph_pass": 3 * args.steps,

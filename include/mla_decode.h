@@ -134,6 +134,27 @@ mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, i
                                 void* out, float* lse, void* stream);
 
 /*
+ * The projections on either side of the latent attention ("absorb + project":
+ * zhaifeiyue "TokenSpeed" notes, DeepSeek-V3 entry).  Per head h, W_UK[h] and W_UV[h]
+ * are the [512 x 128] up-projections of a latent row c (k_nope = c W_UK[h],
+ * v = c W_UV[h]), bf16, stored [H, 512, 128] row-major.  R = B * s_q query rows.
+ *
+ * mla_absorb_q builds the decode's query: q[r, h, 0:512] = W_UK[h] q_nope[r, h] (so that
+ * q . c = q_nope . k_nope), q[r, h, 512:576] = q_rope[r, h] (copied).
+ *   q_nope bf16 [R, H, 128] (16-byte aligned); q_rope bf16 [R, H, 64] (16-byte aligned);
+ *   w_uk bf16 [H, 512, 128] (16-byte aligned); q bf16 [R, H, 576] (16-byte aligned), the
+ *   layout mla_decode reads.
+ * mla_project_out maps the decode's output to the heads' value space:
+ *   y[r, h, :] = out[r, h, :] W_UV[h];  out bf16 [R, H, 512] and w_uv bf16 [H, 512, 128]
+ *   (16-byte aligned), y bf16 [R, H, 128] (4-byte aligned).
+ * Both accumulate in fp32 and round to bf16 (nearest, ties to even).  Argument errors
+ * return before any launch.
+ */
+mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int R, int H, void* q,
+                        void* stream);
+mla_status mla_project_out(const void* out, const void* w_uv, int R, int H, void* y, void* stream);
+
+/*
  * Paged KV append: the write side of the same cache (the step after the decode in the
  * scope table).  The s_q new latent rows of request b -- the draft tokens the decode
  * verifies, counted in seq_lens -- are stored at positions T_b - s_q + i, row

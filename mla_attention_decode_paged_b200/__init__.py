@@ -9,7 +9,8 @@ from __future__ import annotations
 
 from . import _abi
 from ._abi import (MLA_KV_BF16, MLA_KV_E4M3, MlaError, mla_decode_plan, mla_decode_version,
-                   mla_decode_workspace_size, mla_get_device_status, mla_kv_append, mla_split_kv_combine)
+                   mla_decode_workspace_size, mla_get_device_status, mla_kv_append, mla_split_kv_combine,
+                   mla_absorb_q, mla_project_out)
 
 PAGE = 64
 DQK = 576
@@ -105,3 +106,22 @@ def kv_append(ckv_new, kpe_new, rope_cos_sin, kv_pages, block_table, seq_lens, k
                          kv_pages.data_ptr(), kv_dtype, float(kv_scale), block_table.data_ptr(), block_table.shape[1],
                          seq_lens.data_ptr(), B, s_q, kv_pages.shape[0],
                          None if status is None else status.data_ptr(), _stream_ptr(stream)), "mla_kv_append")
+
+
+def absorb_q(q_nope, q_rope, w_uk, q, stream=None):
+    """q[..., 0:512] = W_UK[h] q_nope, q[..., 512:576] = q_rope per head (mla_absorb_q).
+    q_nope bf16 [B, s_q, H, 128], q_rope bf16 [B, s_q, H, 64], w_uk bf16 [H, 512, 128],
+    q bf16 [B, s_q, H, 576]."""
+    H = q_nope.shape[-2]
+    R = q_nope.numel() // (H * 128)
+    _check(mla_absorb_q(q_nope.data_ptr(), q_rope.data_ptr(), w_uk.data_ptr(), R, H, q.data_ptr(),
+                        _stream_ptr(stream)), "mla_absorb_q")
+
+
+def project_out(out, w_uv, y, stream=None):
+    """y = out W_UV[h] per head (mla_project_out): out bf16 [B, s_q, H, 512], w_uv bf16
+    [H, 512, 128], y bf16 [B, s_q, H, 128]."""
+    H = out.shape[-2]
+    R = out.numel() // (H * 512)
+    _check(mla_project_out(out.data_ptr(), w_uv.data_ptr(), R, H, y.data_ptr(), _stream_ptr(stream)),
+           "mla_project_out")

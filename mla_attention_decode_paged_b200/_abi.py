@@ -57,6 +57,10 @@ def lib() -> ctypes.CDLL:
         L.mla_split_kv_combine.restype = I
         L.mla_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.mla_get_device_status.restype = I
+        L.mla_absorb_q.argtypes = [P, P, P, I, I, P, P]
+        L.mla_absorb_q.restype = I
+        L.mla_project_out.argtypes = [P, P, I, I, P, P]
+        L.mla_project_out.restype = I
         L.mla_kv_append.argtypes = [P, P, P, I, P, I, F, P, I, P, I, I, I64, P, P]
         L.mla_kv_append.restype = I
         L.mla_debug_wait_timeout.argtypes = [P, SZ, P]
@@ -105,6 +109,14 @@ def mla_get_device_status(workspace_ptr, stream) -> tuple:
     code = ctypes.c_int(-1)
     rc = lib().mla_get_device_status(workspace_ptr, ctypes.byref(code), stream)
     return rc, code.value
+
+
+def mla_absorb_q(q_nope_ptr, q_rope_ptr, w_uk_ptr, R, H, q_ptr, stream) -> int:
+    return lib().mla_absorb_q(q_nope_ptr, q_rope_ptr, w_uk_ptr, R, H, q_ptr, stream)
+
+
+def mla_project_out(out_ptr, w_uv_ptr, R, H, y_ptr, stream) -> int:
+    return lib().mla_project_out(out_ptr, w_uv_ptr, R, H, y_ptr, stream)
 
 
 def mla_kv_append(ckv_ptr, kpe_ptr, cos_sin_ptr, max_pos, kv_ptr, kv_dtype, kv_scale, block_table_ptr,

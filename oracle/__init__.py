@@ -173,3 +173,19 @@ def kv_append(ckv_bits, kpe_bits, cos_sin, kv, kv_dtype, kv_scale, block_table, 
     if rc != 0:
         raise ValueError("oracle rejected a length or page id")
     return out
+
+
+def absorb_q(q_nope, q_rope, w_uk):
+    """Float64 reference of the query absorption: q[..., :512] = W_UK[h] q_nope (per head),
+    q[..., 512:] = q_rope.  q_nope [..., H, 128], q_rope [..., H, 64], w_uk [H, 512, 128]
+    (any real dtype; computed in float64 with a library matmul)."""
+    qn = np.asarray(q_nope, dtype=np.float64)
+    w = np.asarray(w_uk, dtype=np.float64)
+    qa = np.einsum("hcd,...hd->...hc", w, qn)
+    return np.concatenate([qa, np.asarray(q_rope, dtype=np.float64)], axis=-1)
+
+
+def project_out(out, w_uv):
+    """Float64 reference of the output projection: y = out W_UV[h] per head.
+    out [..., H, 512], w_uv [H, 512, 128]."""
+    return np.einsum("...hc,hcd->...hd", np.asarray(out, dtype=np.float64), np.asarray(w_uv, dtype=np.float64))

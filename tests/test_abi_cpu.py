@@ -118,3 +118,12 @@ def test_kv_append_rejects_bad_arguments_before_any_launch():
     assert call(dt=1, scale=0.0) == _abi.MLA_ERR_INVALID_ARG
     assert call(ckv=256 + 8) == _abi.MLA_ERR_INVALID_ARG  # latent rows need 16-byte alignment
     assert call(status=256 + 2) == _abi.MLA_ERR_INVALID_ARG
+
+
+def test_absorb_and_project_reject_bad_arguments_before_any_launch():
+    assert _abi.mla_absorb_q(None, 256, 256, 4, 16, 256, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_absorb_q(256, 256, 256, 0, 16, 256, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_absorb_q(256, 256, 256, 4, 16, 256 + 8, None) == _abi.MLA_ERR_INVALID_ARG  # q needs 16 B
+    assert _abi.mla_project_out(256, None, 4, 16, 256, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_project_out(256, 256, 4, 0, 256, None) == _abi.MLA_ERR_INVALID_ARG
+    assert _abi.mla_project_out(256, 256, 4, 16, 256 + 2, None) == _abi.MLA_ERR_INVALID_ARG
