@@ -36,7 +36,7 @@ import numpy as np  # noqa: E402
 from mla_attention_decode_paged_b200 import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "agent_spec"
-METRIC = "MLA decode KV-read GB/s (us/call; % of B200 HBM/tensor roofline)"
+METRIC = "MLA decode \u00b5s/call and KV-read GB/s (% of B200 HBM/tensor roofline)"  # value in GB/s; us_per_call beside it
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # B200 datasheet (dense bf16), for context
 KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_sm100.cu"]
