@@ -13,6 +13,8 @@
 // 128-row tensor-core tile) and the result is rounded to bf16 (nearest, ties to even).
 #include <math.h>
 
+#include <algorithm>
+
 #include "mla_common.cuh"
 
 namespace mla {
@@ -25,8 +27,9 @@ constexpr int kKWarps = kAbsorbThreads / 32;
 
 // Y[r, h, n] (row stride y_rs, head stride y_hs) = sum_k X[r, h, k] * B_h[k, n], with
 // X[r, h, k] at x + r * x_rs + h * K + k and B_h[k, n] at w + h * K * N + (B_T ? n * K + k
-// : k * N + n).  One CTA per (32 output columns, head, 16 rows): the weight tile (K x 32,
-// read with 16-byte loads, all in flight together) and the 16 rows go to shared memory;
+// : k * N + n).  A CTA takes 32 output columns of one head and every gridDim.z-th block of
+// 16 rows: the weight tile (K x 32, read once with 16-byte loads, all in flight together)
+// and each block's rows go to shared memory;
 // each warp contracts one eighth of K for the whole 16 x 32 tile (a lane holds a 4 x 4
 // block: 16 independent accumulators), and the eight partial tiles are added in shared
 // memory.
@@ -40,7 +43,7 @@ __global__ void __launch_bounds__(kAbsorbThreads) head_gemm_kernel(const __nv_bf
     __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(absorb_smem);                 // [K][kBN]
     float* xs = reinterpret_cast<float*>(absorb_smem + K * kBN * 2);                    // [K][kRB]
     float* red = xs + K * kRB;                                                          // [kKWarps][kRB][kBN]
-    const int n0 = blockIdx.x * kBN, h = blockIdx.y, r0 = blockIdx.z * kRB;
+    const int n0 = blockIdx.x * kBN, h = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const __nv_bfloat16* wh = w + (int64_t)h * K * N;
     if (B_T) {
@@ -60,59 +63,63 @@ __global__ void __launch_bounds__(kAbsorbThreads) head_gemm_kernel(const __nv_bf
                 *reinterpret_cast<const uint4*>(wh + (int64_t)kk * N + n0 + 8 * c8);
         }
     }
-    // the CTA's 16 rows, transposed to xs[k][row] in fp32
-    for (int e = tid; e < kRB * (K / 8); e += kAbsorbThreads) {
-        const int rr = e / (K / 8), k8 = e % (K / 8);
-        const int r = r0 + rr;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < R) v = *reinterpret_cast<const uint4*>(x + (int64_t)r * x_rs + (int64_t)h * K + 8 * k8);
-        const __nv_bfloat16* pv = reinterpret_cast<const __nv_bfloat16*>(&v);
+    // row blocks blockIdx.z, blockIdx.z + gridDim.z, ...: the weight tile is loaded once
+    for (int r0 = blockIdx.z * kRB; r0 < R; r0 += gridDim.z * kRB) {
+        __syncthreads();  // the previous block's rows and partial tiles are consumed
+        // the block's 16 rows, transposed to xs[k][row] in fp32
+        for (int e = tid; e < kRB * (K / 8); e += kAbsorbThreads) {
+            const int rr = e / (K / 8), k8 = e % (K / 8);
+            const int r = r0 + rr;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r < R) v = *reinterpret_cast<const uint4*>(x + (int64_t)r * x_rs + (int64_t)h * K + 8 * k8);
+            const __nv_bfloat16* pv = reinterpret_cast<const __nv_bfloat16*>(&v);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[(8 * k8 + j) * kRB + rr] = __bfloat162float(pv[j]);
-    }
-    if (rope && blockIdx.x == 0) {
-        // the query's rope part: y[r, h, 512:576] = rope[r, h, :] for this CTA's rows
-        for (int e = tid; e < kRB * 8; e += kAbsorbThreads) {
-            const int rr = e >> 3, p8 = e & 7, r = r0 + rr;
-            if (r < R)
-                *reinterpret_cast<uint4*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + kDv + 8 * p8) =
-                    *reinterpret_cast<const uint4*>(rope + ((int64_t)r * gridDim.y + h) * 64 + 8 * p8);
+            for (int j = 0; j < 8; ++j) xs[(8 * k8 + j) * kRB + rr] = __bfloat162float(pv[j]);
         }
-    }
-    __syncthreads();
-    const int rg = lane >> 3, cg = lane & 7;  // rows 4 rg .. 4 rg + 3, columns 4 cg .. 4 cg + 3
-    float acc[4][4] = {};
-    constexpr int kSlice = K / kKWarps;
+        if (rope && blockIdx.x == 0) {
+            // the query's rope part: y[r, h, 512:576] = rope[r, h, :] for this CTA's rows
+            for (int e = tid; e < kRB * 8; e += kAbsorbThreads) {
+                const int rr = e >> 3, p8 = e & 7, r = r0 + rr;
+                if (r < R)
+                    *reinterpret_cast<uint4*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + kDv + 8 * p8) =
+                        *reinterpret_cast<const uint4*>(rope + ((int64_t)r * gridDim.y + h) * 64 + 8 * p8);
+            }
+        }
+        __syncthreads();
+        const int rg = lane >> 3, cg = lane & 7;  // rows 4 rg .. 4 rg + 3, columns 4 cg .. 4 cg + 3
+        float acc[4][4] = {};
+        constexpr int kSlice = K / kKWarps;
 #pragma unroll 4
-    for (int kk = warp * kSlice; kk < (warp + 1) * kSlice; ++kk) {
-        const float4 xv = *reinterpret_cast<const float4*>(xs + kk * kRB + 4 * rg);
-        const uint2 wb = *reinterpret_cast<const uint2*>(wt + kk * kBN + 4 * cg);
-        const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.x));
-        const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.y));
-        const float xr[4] = {xv.x, xv.y, xv.z, xv.w}, wc[4] = {w01.x, w01.y, w23.x, w23.y};
+        for (int kk = warp * kSlice; kk < (warp + 1) * kSlice; ++kk) {
+            const float4 xv = *reinterpret_cast<const float4*>(xs + kk * kRB + 4 * rg);
+            const uint2 wb = *reinterpret_cast<const uint2*>(wt + kk * kBN + 4 * cg);
+            const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.x));
+            const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.y));
+            const float xr[4] = {xv.x, xv.y, xv.z, xv.w}, wc[4] = {w01.x, w01.y, w23.x, w23.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xr[i], wc[j], acc[i][j]);
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(red + (warp * kRB + 4 * rg + i) * kBN + 4 * cg) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        __syncthreads();
+        // the eight partial tiles, added in warp order (a fixed order: deterministic)
+        for (int o = tid; o < kRB * kBN / 2; o += kAbsorbThreads) {
+            const int rr = o / (kBN / 2), c = 2 * (o % (kBN / 2));
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xr[i], wc[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(red + (warp * kRB + 4 * rg + i) * kBN + 4 * cg) =
-            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    __syncthreads();
-    // the eight partial tiles, added in warp order (a fixed order: deterministic)
-    for (int o = tid; o < kRB * kBN / 2; o += kAbsorbThreads) {
-        const int rr = o / (kBN / 2), c = 2 * (o % (kBN / 2));
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int q = 0; q < kKWarps; ++q) {
-            s0 += red[(q * kRB + rr) * kBN + c];
-            s1 += red[(q * kRB + rr) * kBN + c + 1];
+            for (int q = 0; q < kKWarps; ++q) {
+                s0 += red[(q * kRB + rr) * kBN + c];
+                s1 += red[(q * kRB + rr) * kBN + c + 1];
+            }
+            const int r = r0 + rr;
+            if (r < R)
+                *reinterpret_cast<__nv_bfloat162*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + n0 + c) =
+                    __floats2bfloat162_rn(s0, s1);
         }
-        const int r = r0 + rr;
-        if (r < R)
-            *reinterpret_cast<__nv_bfloat162*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + n0 + c) =
-                __floats2bfloat162_rn(s0, s1);
     }
 }
 
@@ -125,7 +132,9 @@ cudaError_t launch_head_gemm(const __nv_bfloat16* x, int64_t x_rs, const __nv_bf
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
     }
-    head_gemm_kernel<B_T, K, N><<<dim3(N / kBN, H, (R + kRB - 1) / kRB), kAbsorbThreads, kSmem, st>>>(
+    // at most four CTAs share a (head, column tile): each reads the weight tile once
+    const int zblocks = std::min((R + kRB - 1) / kRB, 4);
+    head_gemm_kernel<B_T, K, N><<<dim3(N / kBN, H, zblocks), kAbsorbThreads, kSmem, st>>>(
         x, x_rs, w, y, y_rs, y_hs, R, rope);
     return cudaGetLastError();
 }
