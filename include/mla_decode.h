@@ -6,9 +6,9 @@
  * token: a 512-wide c_kv plus a decoupled 64-wide RoPE key, 576 values in all
  * ["TokenSpeed" related-work notes (zhaifeiyue.github.io), DeepSeek-V3 entry: 512-dim
  * latent KV; llm-atlas "Inference systems", 22 DeepSeek V2->V3: RoPE part decoupled].
- * Decode runs in that latent space ("absorb + project", same entry): the caller has
- * already multiplied the no-RoPE query through W_UK, so q is 576 wide, and multiplies
- * the 512-wide output through W_UV afterwards.  The s_q speculative query tokens of a
+ * Decode runs in that latent space ("absorb + project", same entry): the no-RoPE query
+ * is multiplied through W_UK first, so q is 576 wide, and the 512-wide output through
+ * W_UV afterwards (mla_absorb_q and mla_project_out below, or the caller's own GEMMs).  The s_q speculative query tokens of a
  * request and its H heads are folded into one row axis of M = s_q * H rows, row
  * m = i * H + h, all attending to the same cached rows ("TokenSpeed" launch digest
  * (cvshuo.com), MLA kernel paragraphs: the query-sequence axis is folded into the
