@@ -138,12 +138,15 @@ class ClockSampler:
 
 
 def oracle_sample(wl, n_req=None):
-    """Time the oracle on n_req requests x a head subset giving 16 rows (one oracle row
-    block) per request; returns (seconds for the full workload, extrapolated by rows and
+    """Time the oracle on n_req requests x a head subset (16-row blocks, enough of them to
+    give every host core one); returns (seconds for the full workload, extrapolated by rows and
     by the sampled requests' share of cache tokens, threads used, description)."""
     import oracle
-    heads = list(range(max(1, min(wl.H, 16 // wl.s_q))))
     reqs = list(range(wl.B if n_req is None else max(1, min(wl.B, n_req))))
+    # enough 16-row blocks per request that every host core has one (the oracle runs one
+    # OpenMP task per request and 16-row block)
+    blocks = max(1, -(-len(os.sched_getaffinity(0)) // len(reqs)))
+    heads = list(range(max(1, min(wl.H, 16 * blocks // wl.s_q))))
     rows_s = wl.s_q * len(heads)
     t0 = time.perf_counter()
     oracle.mla_decode(wl.q[reqs][:, :, heads], wl.kv, wl.kv_dtype, wl.kv_scale, wl.block_table[reqs],
@@ -155,6 +158,30 @@ def oracle_sample(wl, n_req=None):
     desc = (f"oracle on {len(reqs)} of {wl.B} requests x {len(heads)} head(s) x {wl.s_q} drafts = {rows_s} of "
             f"{wl.spec.M} rows per request ({dt:.2f} s), scaled by rows and cache tokens to the full workload")
     return full, cores, desc
+
+
+def oracle_baseline(wl, target_s=10.0, cap_s=30.0):
+    """The oracle timed on about target_s seconds of CPU work (never past cap_s): a pilot
+    sample sizes the number of requests, then the sample is repeated until target_s is
+    reached.  Returns (seconds for the full workload, threads used, description)."""
+    t0 = time.perf_counter()
+    pilot, _, _ = oracle_sample(wl, 1)
+    pilot_s = time.perf_counter() - t0
+    # the pilot ran one request's 16-row sample; a run over n requests costs about n times it
+    per_req = max(pilot_s, 1e-3)
+    n_req = int(max(1, min(wl.B, target_s / per_req)))
+    runs, total, full = 0, 0.0, []
+    cores, desc = 0, ""
+    while True:
+        t1 = time.perf_counter()
+        f, cores, desc = oracle_sample(wl, n_req)
+        total += time.perf_counter() - t1
+        full.append(f)
+        runs += 1
+        if total >= target_s or total + total / runs > cap_s:
+            break
+    return (sum(full) / len(full), cores,
+            f"{desc}; {runs} run(s), {total:.1f} s of CPU time in all, after a one-request pilot")
 
 
 def run_reference(args):
@@ -494,7 +521,7 @@ def run_ours(args):
             "gpu_launches_graph_pass": 3 * args.steps,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        full_s, cores, desc = oracle_sample(wl)
+        full_s, cores, desc = oracle_baseline(wl)
         line["cpu_baseline"] = {"value": kvb / full_s / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": desc}
     if rank == 0:
