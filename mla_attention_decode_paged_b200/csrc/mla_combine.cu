@@ -6,7 +6,8 @@
 //     L = log2 sum_j 2^lse2_j,   out = sum_j 2^(lse2_j - L) * o_j,   lse = L * ln 2,
 // the reduction pass of split-KV decoding ["Faster kernels, slower engine", 7.1 Gluon
 // MLA decode].  A split in which a row sees no token has lse2_j = -inf and o_j = 0, so
-// it drops out.  The kernel reads every partial once; it is bound by that read.
+// it drops out.  The kernel reads every partial once; it is bound by that read.  A
+// request without tokens has no split at all; its rows are written here, as NaN.
 #include <string.h>
 
 #include "mla_decode_params.cuh"
