@@ -78,11 +78,14 @@ size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
 
 /*
  * Split planner (one small kernel on `stream`).  From seq_lens[B] (device int32) it
- * partitions the pages of all requests into equal contiguous shares, one share per
- * group of SM pairs, cutting requests into splits where a share ends.  The plan is
- * written into `workspace` and is valid for every later mla_decode of the same
- * seq_lens, B, s_q and H (e.g. all layers of one decode step).  num_sms as above; a
- * smaller value gives fewer, longer splits (1 = no splits at all).
+ * partitions the pages of all requests, laid end to end, into G equal contiguous shares
+ * (G = num_sms / row blocks, a row block being 64 folded query rows), one share per
+ * group of scan CTAs (one CTA per row block), cutting requests into splits where a
+ * share ends.  The plan is written into `workspace` and is valid for every later
+ * mla_decode of the same seq_lens, B, s_q and H (e.g. all layers of one decode step).
+ * num_sms as above; a smaller value gives fewer, longer splits (1 = no splits at all);
+ * a plan made for more groups than the device runs at once is refused by the decode
+ * (device status MLA_ERR_PLAN_MISMATCH).
  */
 mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, int H, int num_sms,
                            void* workspace, size_t ws_bytes, void* stream);
