@@ -71,8 +71,9 @@ typedef enum { MLA_KV_BF16 = 0, MLA_KV_E4M3 = 1 } mla_kv_dtype;
 /*
  * Bytes of workspace a plan + decode of this shape needs (host, pure).
  * num_sms: SM count the split plan is made for; 0 = the current device's.
- * Returns 0 for an unsupported shape (B, s_q, H <= 0, or s_q * H > 65536) or for a
- * num_sms that would make more than 1023 groups.
+ * Returns 0 for an unsupported shape (B, s_q, H <= 0, or s_q * H > 65536), for a
+ * num_sms that would make more than 1023 groups, or for a batch too large for the
+ * planner's shared memory (more than about 12,000 requests).
  */
 size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
 
@@ -184,6 +185,43 @@ mla_status mla_kv_append(const void* ckv_new, const void* kpe_new, const float* 
                          void* kv_pages, int kv_dtype, float kv_scale, const int32_t* block_table,
                          int max_pages_per_req, const int32_t* seq_lens, int B, int s_q, int64_t num_pages,
                          int32_t* status, void* stream);
+
+/*
+ * Long-prefix MLA prefill: the second workload shape on the same cache (the prefill
+ * workloads "with a long-prefix KV cache" of the "TokenSpeed" launch digest
+ * (cvshuo.com), MLA kernel paragraphs).  Request b adds a chunk of `chunk` query tokens
+ * whose latent rows are already its last `chunk` cache rows (seq_lens counts them, as it
+ * counts the drafts of a decode): chunk token i sees cached tokens t <= T_b - chunk + i.
+ * Each row's result is the decode's: out = softmax_t(scale q . KV_t) KV_t[0:512] and
+ * lse = ln sum_t exp(scale q . KV_t).
+ *   q           bf16 [B, chunk, H, 576], absorbed as for mla_decode
+ *   kv_pages, kv_dtype, kv_scale, block_table, max_pages_per_req, num_pages, scale:
+ *               as for mla_decode
+ *   seq_lens    int32 [B] (4-byte aligned), chunk <= T_b <= max_pages_per_req * 64
+ *   workspace   at least mla_prefill_workspace_size(B, chunk, H, max_pages_per_req, 0)
+ *               bytes, 256-byte aligned, owned by the caller
+ *   out         bf16 [B, chunk, H, 512];  lse  fp32 [B, chunk, H], natural log
+ * The chunk runs on the decode path.  It is cut into sub-chunks of
+ * d = mla_prefill_sub_chunk(chunk, H) tokens (d divides chunk, d * H <= 256 rows), and
+ * sub-chunk j of request b is scanned as a decode request with seq_len
+ * T_b - chunk + (j + 1) d and b's block-table row: its draft k is chunk token j d + k and
+ * sees exactly the chunk's causal prefix.  q, out and lse need no copy (they are the
+ * decode's arrays for B * chunk / d requests of d drafts).  A small kernel writes those
+ * lengths and block-table rows into the workspace, then the planner, the split scan and
+ * the combine run, all on `stream`; nothing is allocated or synchronised.  A request with
+ * T_b < chunk or T_b > max_pages_per_req * 64 sets the device status MLA_ERR_DEVICE_OOB
+ * and its rows come out NaN.
+ * mla_prefill_sub_chunk (host, pure) returns d: the divisor of `chunk` with d * H <= 256
+ * that needs the fewest 64-row blocks, (chunk / d) * ceil(d H / 64), ties to the larger;
+ * 0 if chunk <= 0, H <= 0 or H > 256.  mla_prefill_workspace_size returns 0 for an
+ * unsupported shape (as mla_decode_workspace_size, for B * chunk / d requests).
+ */
+int mla_prefill_sub_chunk(int chunk, int H);
+size_t mla_prefill_workspace_size(int B, int chunk, int H, int max_pages_per_req, int num_sms);
+mla_status mla_prefill(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,
+                       const int32_t* block_table, int max_pages_per_req, const int32_t* seq_lens,
+                       int B, int chunk, int H, int64_t num_pages, float scale, void* workspace,
+                       size_t ws_bytes, void* out, float* lse, void* stream);
 
 /*
  * Test and debugging aid for the device-side failure detection (no counterpart on the

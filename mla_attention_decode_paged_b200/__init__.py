@@ -10,7 +10,8 @@ from __future__ import annotations
 from . import _abi
 from ._abi import (MLA_KV_BF16, MLA_KV_E4M3, MlaError, mla_decode_plan, mla_decode_version,
                    mla_decode_workspace_size, mla_get_device_status, mla_kv_append, mla_split_kv_combine,
-                   mla_absorb_q, mla_project_out)
+                   mla_absorb_q, mla_project_out, mla_prefill, mla_prefill_sub_chunk,
+                   mla_prefill_workspace_size)
 
 PAGE = 64
 DQK = 576
@@ -27,6 +28,15 @@ def _stream_ptr(stream):
 def _check(rc, what):
     if rc != 0:
         raise MlaError(rc, what)
+
+
+def _kv_dtype(kv_pages):
+    import torch
+    if kv_pages.dtype == torch.bfloat16:
+        return MLA_KV_BF16
+    if kv_pages.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return MLA_KV_E4M3
+    raise TypeError(f"unsupported cache dtype {kv_pages.dtype}")
 
 
 def workspace_bytes(B: int, s_q: int, H: int, num_sms: int = 0) -> int:
@@ -64,12 +74,7 @@ def decode(q, kv_pages, block_table, seq_lens, scale: float, causal: bool, works
     import torch
     B, s_q, H, d = q.shape
     assert d == DQK and q.dtype == torch.bfloat16 and q.is_contiguous()
-    if kv_pages.dtype == torch.bfloat16:
-        kv_dtype = MLA_KV_BF16
-    elif kv_pages.dtype in (torch.uint8, torch.float8_e4m3fn):
-        kv_dtype = MLA_KV_E4M3
-    else:
-        raise TypeError(f"unsupported cache dtype {kv_pages.dtype}")
+    kv_dtype = _kv_dtype(kv_pages)
     assert kv_pages.is_contiguous() and kv_pages.shape[1:] == (PAGE, DQK)
     assert block_table.dtype == torch.int32 and block_table.is_contiguous()
     assert seq_lens.dtype == torch.int32 and out.dtype == torch.bfloat16 and lse.dtype == torch.float32
@@ -125,3 +130,36 @@ def project_out(out, w_uv, y, stream=None):
     R = out.numel() // (H * 512)
     _check(mla_project_out(out.data_ptr(), w_uv.data_ptr(), R, H, y.data_ptr(), _stream_ptr(stream)),
            "mla_project_out")
+
+
+def prefill_workspace_bytes(B: int, chunk: int, H: int, max_pages: int, num_sms: int = 0) -> int:
+    n = mla_prefill_workspace_size(B, chunk, H, max_pages, num_sms)
+    if n == 0:
+        raise MlaError(_abi.MLA_ERR_UNSUPPORTED, "mla_prefill_workspace_size")
+    return n
+
+
+def alloc_prefill_workspace(B: int, chunk: int, H: int, max_pages: int, device=None):
+    """A zero-filled uint8 CUDA tensor large enough for mla_prefill."""
+    import torch
+    return torch.zeros(prefill_workspace_bytes(B, chunk, H, max_pages), dtype=torch.uint8, device=device or "cuda")
+
+
+def prefill(q, kv_pages, block_table, seq_lens, scale: float, workspace, out, lse, kv_scale: float = 1.0,
+            stream=None):
+    """Enqueue mla_prefill: the chunk of q.shape[1] query tokens of each request, whose rows
+    are the request's last cache rows, attends causally to its paged cache.  q bf16
+    [B, chunk, H, 576]; out bf16 [B, chunk, H, 512]; lse float32 [B, chunk, H]; the other
+    arguments as for ``decode``; ``workspace`` from ``alloc_prefill_workspace``."""
+    import torch
+    B, chunk, H, d = q.shape
+    assert d == DQK and q.dtype == torch.bfloat16 and q.is_contiguous()
+    kv_dtype = _kv_dtype(kv_pages)
+    assert kv_pages.is_contiguous() and kv_pages.shape[1:] == (PAGE, DQK)
+    assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+    assert seq_lens.dtype == torch.int32 and out.dtype == torch.bfloat16 and lse.dtype == torch.float32
+    assert out.is_contiguous() and lse.is_contiguous()
+    _check(mla_prefill(q.data_ptr(), kv_pages.data_ptr(), kv_dtype, float(kv_scale), block_table.data_ptr(),
+                       int(block_table.shape[1]), seq_lens.data_ptr(), B, chunk, H, int(kv_pages.shape[0]),
+                       float(scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(), lse.data_ptr(),
+                       _stream_ptr(stream)), "mla_prefill")

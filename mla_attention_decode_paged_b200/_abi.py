@@ -65,6 +65,12 @@ def lib() -> ctypes.CDLL:
         L.mla_kv_append.restype = I
         L.mla_debug_wait_timeout.argtypes = [P, SZ, P]
         L.mla_debug_wait_timeout.restype = I
+        L.mla_prefill_sub_chunk.argtypes = [I, I]
+        L.mla_prefill_sub_chunk.restype = I
+        L.mla_prefill_workspace_size.argtypes = [I, I, I, I, I]
+        L.mla_prefill_workspace_size.restype = SZ
+        L.mla_prefill.argtypes = [P, P, I, F, P, I, P, I, I, I, I64, F, P, SZ, P, P, P]
+        L.mla_prefill.restype = I
         L.mla_decode_version.argtypes = []
         L.mla_decode_version.restype = ctypes.c_char_p
         _lib = L
@@ -123,6 +129,20 @@ def mla_kv_append(ckv_ptr, kpe_ptr, cos_sin_ptr, max_pos, kv_ptr, kv_dtype, kv_s
                   max_pages_per_req, seq_lens_ptr, B, s_q, num_pages, status_ptr, stream) -> int:
     return lib().mla_kv_append(ckv_ptr, kpe_ptr, cos_sin_ptr, max_pos, kv_ptr, kv_dtype, kv_scale, block_table_ptr,
                                max_pages_per_req, seq_lens_ptr, B, s_q, num_pages, status_ptr, stream)
+
+
+def mla_prefill_sub_chunk(chunk: int, H: int) -> int:
+    return int(lib().mla_prefill_sub_chunk(chunk, H))
+
+
+def mla_prefill_workspace_size(B: int, chunk: int, H: int, max_pages_per_req: int, num_sms: int = 0) -> int:
+    return int(lib().mla_prefill_workspace_size(B, chunk, H, max_pages_per_req, num_sms))
+
+
+def mla_prefill(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_pages_per_req, seq_lens_ptr, B, chunk, H,
+                num_pages, scale, workspace_ptr, ws_bytes, out_ptr, lse_ptr, stream) -> int:
+    return lib().mla_prefill(q_ptr, kv_ptr, kv_dtype, kv_scale, block_table_ptr, max_pages_per_req, seq_lens_ptr,
+                             B, chunk, H, num_pages, scale, workspace_ptr, ws_bytes, out_ptr, lse_ptr, stream)
 
 
 def mla_debug_wait_timeout(workspace_ptr, ws_bytes, stream) -> int:

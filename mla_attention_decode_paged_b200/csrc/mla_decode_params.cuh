@@ -23,7 +23,13 @@ struct DecodeParams {
     float out_scale;            // kv_scale for e4m3 (values are e4m3 * kv_scale), 1 for bf16
 };
 
-mla_status launch_decode_simt(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
+// Dynamic shared memory of the plan kernel (one CTA) for B requests and G groups, and
+// the most the planner takes: shapes beyond it are unsupported.
+inline size_t plan_shared_bytes(int B, int G) {
+    return sizeof(int64_t) * (2 * ((size_t)B + 1) + (size_t)G + 2 + 16);
+}
+constexpr size_t kPlanMaxSharedBytes = 200 * 1024;
+
 mla_status launch_decode_sm100(const DecodeParams& p, int kv_dtype, cudaStream_t stream);
 // One CTA that runs the scan kernel's bounded wait on a barrier nothing arrives at (20 ms
 // limit) and so sets the timeout status in the workspace header.

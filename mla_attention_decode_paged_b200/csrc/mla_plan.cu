@@ -242,7 +242,7 @@ extern "C" size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms) 
         if (num_sms <= 0) return 0;
     }
     WsLayout L = make_layout(B, s_q, H, num_groups_for(num_sms, num_row_blocks(s_q, H)));
-    if (L.num_groups > kMaxGroups) return 0;
+    if (L.num_groups > kMaxGroups || plan_shared_bytes(B, L.num_groups) > kPlanMaxSharedBytes) return 0;
     return (size_t)L.total;
 }
 
@@ -258,8 +258,8 @@ extern "C" mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, i
     WsLayout L = make_layout(B, s_q, H, num_groups_for(num_sms, num_row_blocks(s_q, H)));
     if (L.num_groups > kMaxGroups) return MLA_ERR_UNSUPPORTED;
     if ((int64_t)ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
-    const size_t smem = sizeof(int64_t) * (2 * ((size_t)B + 1) + (size_t)L.num_groups + 2 + 16);
-    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+    const size_t smem = plan_shared_bytes(B, L.num_groups);
+    if (smem > kPlanMaxSharedBytes) return MLA_ERR_UNSUPPORTED;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;

@@ -114,6 +114,17 @@ def mla_decode(q_bits, kv, kv_dtype, kv_scale, block_table, seq_lens, scale, cau
     return out, lse
 
 
+def mla_prefill(q_bits, kv, kv_dtype, kv_scale, block_table, seq_lens, scale, page=PAGE):
+    """Float64 reference of long-prefix chunked prefill over the paged cache (the prefill
+    workloads with a long-prefix KV cache of the "TokenSpeed" launch digest, MLA kernel
+    paragraphs).  The chunk of C = q_bits.shape[1] query tokens of request b are its last C
+    cache rows (seq_lens counts them); chunk token i, at position T_b - C + i, sees the
+    cached tokens t <= T_b - C + i.  That is the visibility rule of the decode definition
+    with s_q = C under the causal flag, so the result is that definition evaluated with
+    s_q = C.  Returns (out float64 [B, C, H, 512], lse float64 [B, C, H])."""
+    return mla_decode(q_bits, kv, kv_dtype, kv_scale, block_table, seq_lens, scale, True, page=page)
+
+
 def combine(outs, lses):
     """LSE-weighted combination of partial results: outs [n, ..., 512], lses [n, ...]."""
     lib = _load()

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import mla_attention_decode_paged_b200 as mla
@@ -127,3 +128,53 @@ def test_absorb_and_project_reject_bad_arguments_before_any_launch():
     assert _abi.mla_project_out(256, None, 4, 16, 256, None) == _abi.MLA_ERR_INVALID_ARG
     assert _abi.mla_project_out(256, 256, 4, 0, 256, None) == _abi.MLA_ERR_INVALID_ARG
     assert _abi.mla_project_out(256, 256, 4, 16, 256 + 2, None) == _abi.MLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("chunk,H,d", [(24, 16, 12), (1000, 16, 8), (7, 128, 1), (64, 8, 32), (4096, 128, 2),
+                                       (16, 16, 16), (1, 1, 1), (256, 1, 256), (5, 300, 0), (0, 16, 0)])
+def test_prefill_sub_chunk_examples(chunk, H, d):
+    assert mla.mla_prefill_sub_chunk(chunk, H) == d
+
+
+def test_prefill_sub_chunk_is_the_cheapest_divisor():
+    rng = np.random.default_rng(0)
+    for _ in range(300):
+        chunk, H = int(rng.integers(1, 3000)), int(rng.integers(1, 257))
+        d = mla.mla_prefill_sub_chunk(chunk, H)
+        divs = [e for e in range(1, chunk + 1) if chunk % e == 0 and e * H <= 256]
+        cost = {e: (chunk // e) * -(-(e * H) // 64) for e in divs}
+        assert d == max(e for e in divs if cost[e] == min(cost.values())), (chunk, H, d)
+
+
+def test_prefill_workspace_holds_the_decode_workspace_and_the_copied_tables():
+    B, chunk, H, mp = 3, 24, 16, 40
+    d = mla.mla_prefill_sub_chunk(chunk, H)
+    n = chunk // d
+    ws = mla.mla_prefill_workspace_size(B, chunk, H, mp, 148)
+    assert ws % 256 == 0
+    assert ws >= mla.mla_decode_workspace_size(B * n, d, H, 148) + 4 * B * n * (mp + 1)
+    assert mla.mla_prefill_workspace_size(B, chunk, 300, mp, 148) == 0
+    assert mla.mla_prefill_workspace_size(0, chunk, H, mp, 148) == 0
+    assert mla.mla_prefill_workspace_size(B, chunk, H, 0, 148) == 0
+    # more sub-chunk requests than the planner takes
+    assert mla.mla_prefill_workspace_size(20000, 7, 64, mp, 148) == 0
+
+
+def test_prefill_rejects_bad_arguments_before_any_launch():
+    ok = dict(q=256, kv=256, dt=0, ks=1.0, bt=256, mp=4, sl=256, B=2, chunk=8, H=16, P=8, scale=0.07, ws=256,
+              wsb=1 << 30, out=256, lse=256)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return _abi.mla_prefill(*a.values(), None)
+    assert call(q=None) == _abi.MLA_ERR_INVALID_ARG
+    assert call(sl=None) == _abi.MLA_ERR_INVALID_ARG
+    assert call(chunk=0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(P=0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == _abi.MLA_ERR_INVALID_ARG
+    assert call(dt=3) == _abi.MLA_ERR_UNSUPPORTED
+    assert call(dt=1, ks=-1.0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(H=300) == _abi.MLA_ERR_UNSUPPORTED
+    assert call(q=256 + 8) == _abi.MLA_ERR_INVALID_ARG
+    assert call(sl=256 + 2) == _abi.MLA_ERR_INVALID_ARG
+    assert call(ws=256 + 16) == _abi.MLA_ERR_INVALID_ARG
