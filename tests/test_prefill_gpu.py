@@ -80,3 +80,20 @@ def test_prefill_rejects_a_small_workspace():
     with pytest.raises(mla.MlaError) as e:
         mla.prefill(q, kv, bt, sl, wl.scale, ws, out, lse)
     assert e.value.code == _abi.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_bench_size_prefill_on_sampled_rows():
+    """The prefill bench.py times (one request, chunk 1024 x 16 heads ending a 65,536-token
+    cache), compared on sampled rows: chunk tokens 0, 511, 1023 (first and last head),
+    each against a one-token oracle decode over its visible prefix."""
+    import oracle
+    C, H, T = 1024, 16, 65536
+    wl = _workload(1, C, H, [T], W.KV_BF16, seed=21)
+    out, lse, code = _run_prefill(wl)
+    assert code == 0
+    heads = [0, H - 1]
+    for i in (0, 511, C - 1):
+        ref_out, ref_lse = oracle.mla_decode(wl.q[:, i:i + 1][:, :, heads], wl.kv, wl.kv_dtype, wl.kv_scale,
+                                             wl.block_table, np.array([T - C + i + 1], np.int32), wl.scale, False)
+        pu.check_close(out[:, i:i + 1][:, :, heads], lse[:, i:i + 1][:, :, heads], ref_out, ref_lse, wl.kv_dtype,
+                       what=f"bench-size prefill token {i}")
