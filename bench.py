@@ -10,6 +10,12 @@ rows the decode must read, summed over ranks, divided by the slowest rank's devi
 time); us_per_call is the per-step latency.  The L2 (126 MB) is flushed by a 256 MB
 write between timed steps, outside the timed events.
 
+Beside the step the line carries, each timed on its own with CUDA events and the L2
+flushed before every call: the paged KV append of the drafts' rows (kv_append), the
+projections either side of the latent attention (absorb_project), and a long-prefix
+chunked prefill on the same path (prefill: one request, 1024 query tokens x 16 heads at
+the end of a 65,536-token cache).
+
 Multi-GPU (torchrun): every rank decodes its own replica of the workload (requests are
 independent; there is no data-path collective), time = max over ranks, scaling weak.
 
