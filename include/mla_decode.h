@@ -31,9 +31,10 @@
  *  - Pointers are DEVICE pointers unless marked host.  All arrays are dense,
  *    row-major, and start on a 16-byte boundary (the cache and q on 128 bytes).
  *  - The caller owns every buffer, including the workspace; nothing is retained after
- *    a call returns.  mla_decode_plan / mla_decode / mla_split_kv_combine never
- *    allocate, free or synchronise: they enqueue work on `stream` (a cudaStream_t,
- *    0 = legacy default stream) and return.
+ *    a call returns.  mla_decode_plan / mla_decode / mla_split_kv_combine and the other
+ *    compute entry points (mla_prefill, mla_kv_append, mla_absorb_q, mla_project_out)
+ *    never allocate, free or synchronise: they enqueue work on `stream` (a
+ *    cudaStream_t, 0 = legacy default stream) and return.
  *  - Errors are return codes; nothing is thrown across the ABI.  Arguments are
  *    checked on the host before anything is enqueued.  Conditions only the device can
  *    see (a page id outside [0, num_pages), seq_len outside [1, max_pages * 64], or

@@ -46,9 +46,9 @@ def test_no_prefix_equals_library_causal_attention():
     ref = F.scaled_dot_product_attention(q, kv.expand(H, C, 576), kv[:, :512].expand(H, C, 512), is_causal=True,
                                          scale=wl.scale)
     assert np.abs(out[0].transpose(1, 0, 2) - ref.numpy()).max() < 1e-12
-    # lse of the first token: it sees one key only
-    s00 = wl.scale * float(q[:, 0] @ kv[0]) if H == 1 else wl.scale * (q[:, 0] @ kv[0]).numpy()
-    assert np.abs(lse[0, 0] - s00).max() < 1e-12
+    # the first token sees one key only: its lse is that key's score
+    s0 = wl.scale * (q[:, 0] @ kv[0]).numpy()  # [H]
+    assert np.abs(lse[0, 0] - s0).max() < 1e-12
 
 
 def test_every_chunk_row_equals_a_one_token_decode_over_its_prefix():
@@ -75,8 +75,9 @@ def test_planted_key_is_seen_from_its_own_token_on():
     t0 = prefix + k
     pg, off = int(wl.block_table[0, t0 // PAGE]), t0 % PAGE
     qf = W.bf16_bits_to_float32(wl.q[0]).astype(np.float64)
-    # the planted row: a multiple of the first query row (large score for every head whose
-    # query is correlated with it); head 0 of every chunk row gets q = that row
+    # the planted row is 4 sign(q) over the latent columns of one query row (rope part 0), and
+    # head 0 of every chunk row gets q = sign(that row): its score with the planted row is
+    # 4 * 512 * scale (about 148), far above every other score
     row = np.zeros(576, np.float32)
     row[:512] = 4.0 * np.sign(qf[0, 0, :512])
     wl.kv[pg, off] = W._bf16_bits(row)
