@@ -51,6 +51,10 @@ def test_workspace_size_is_pure_host_and_grows_with_shape():
     assert b >= (16 + 37) * 2 * 128 * 512 * 4
     assert mla.mla_decode_workspace_size(0, 4, 16, 148) == 0
     assert mla.mla_decode_workspace_size(4, -1, 16, 148) == 0
+    # the planner keeps two int64 per request in shared memory (at most 200 KB): beyond about
+    # 12,700 requests the shape is unsupported, and the size says so
+    assert mla.mla_decode_workspace_size(12000, 1, 16, 148) > 0
+    assert mla.mla_decode_workspace_size(13000, 1, 16, 148) == 0
 
 
 def _decode_args(**kw):
