@@ -59,7 +59,7 @@ def test_edge_cases(kw, num_sms):
 
 
 def test_many_short_requests():
-    """More requests than the planner has threads: every planner loop runs several rounds."""
+    """More requests than the planner has threads: every planner loop makes several passes."""
     _case("agent_spec", 0, B=300, s_q=1, H=16, seq=("uniform", 1, 1500))
 
 
