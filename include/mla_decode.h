@@ -188,9 +188,9 @@ mla_status mla_kv_append(const void* ckv_new, const void* kpe_new, const float* 
                          int32_t* status, void* stream);
 
 /*
- * Long-prefix MLA prefill: the second workload shape on the same cache (the prefill
- * workloads "with a long-prefix KV cache" of the "TokenSpeed" launch digest
- * (cvshuo.com), MLA kernel paragraphs).  Request b adds a chunk of `chunk` query tokens
+ * Long-prefix MLA prefill: the second workload shape on the same cache (prefill over a
+ * cache that already holds a long prefix is the other MLA workload of the "TokenSpeed"
+ * launch digest (cvshuo.com), MLA kernel paragraphs).  Request b adds a chunk of `chunk` query tokens
  * whose latent rows are already its last `chunk` cache rows (seq_lens counts them, as it
  * counts the drafts of a decode): chunk token i sees cached tokens t <= T_b - chunk + i.
  * Each row's result is the decode's: out = softmax_t(scale q . KV_t) KV_t[0:512] and
