@@ -1,8 +1,9 @@
 // mla_prefill.cu -- long-prefix MLA prefill: a chunk of C new query tokens per request
 // attends causally to the request's paged latent cache, whose last C rows are the chunk's
 // own (prefill over a cache that already holds a long prefix is one of the two MLA
-// workloads of the "TokenSpeed" launch digest (cvshuo.com), MLA kernel paragraphs).  Token i of the chunk of request b sits at
-// position T_b - C + i and sees cached tokens t <= T_b - C + i.
+// workloads of the "TokenSpeed" launch digest (cvshuo.com), MLA kernel paragraphs).
+// Token i of the chunk of request b sits at position T_b - C + i and sees cached tokens
+// t <= T_b - C + i.
 //
 // That is the decode's causal rule with s_q = C, so the prefill runs on the decode path.
 // The chunk is cut into n = C / d sub-chunks of d tokens, d * H <= 256 rows each; each
