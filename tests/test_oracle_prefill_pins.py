@@ -112,3 +112,19 @@ def test_sub_chunks_as_decode_requests_reproduce_the_prefill(C, d, kv_dtype):
     o2, l2 = oracle.mla_decode(q_x, wl.kv, wl.kv_dtype, wl.kv_scale, bt_x, lens_x, wl.scale, True)
     assert np.array_equal(o2.reshape(out.shape), out)
     assert np.array_equal(l2.reshape(lse.shape), lse)
+
+
+def test_gpu_prefill_cases_would_reject_a_kernel_without_the_chunk_mask():
+    """Negative control for the GPU prefill cases: the same inputs with the chunk's causal
+    triangle dropped (every chunk token sees the whole chunk) fail the parity gate."""
+    from tests import parity_util as pu
+    from tests.test_prefill_gpu import PREFILL_CASES
+    for B, C, H, lens, kv_dtype in PREFILL_CASES:
+        name = "agent_spec" if kv_dtype == W.KV_BF16 else "fp8_batch"
+        wl = W.make_workload(name, B=B, s_q=C, H=H, seq_lens=lens, seed=11)
+        ref = _prefill(wl)
+        no_mask = oracle.mla_decode(wl.q, wl.kv, wl.kv_dtype, wl.kv_scale, wl.block_table, wl.seq_lens, wl.scale,
+                                    False)
+        with pytest.raises(AssertionError):
+            pu.check_close(*no_mask, *ref, kv_dtype)
+

@@ -38,13 +38,16 @@ def _run_prefill(wl):
     return out.float().cpu().numpy(), lse.cpu().numpy(), mla.device_status(ws)
 
 
-@pytest.mark.parametrize("B,C,H,lens,kv_dtype", [
+PREFILL_CASES = [
     (2, 24, 16, [300, 1000], W.KV_BF16),          # d = 12: three 64-row blocks per sub-chunk
     (1, 7, 128, [137], W.KV_BF16),                # d = 1: seven one-token sub-chunks of 128 rows
     (3, 64, 8, [64, 500, 2100], W.KV_BF16),       # d = 32; the first request has no prefix
     (2, 32, 16, [40, 3000], W.KV_E4M3),           # e4m3 cache
     (1, 200, 16, [2000], W.KV_BF16),              # d = 8: 25 sub-chunks
-])
+]
+
+
+@pytest.mark.parametrize("B,C,H,lens,kv_dtype", PREFILL_CASES)
 def test_prefill_matches_the_oracle(B, C, H, lens, kv_dtype):
     import oracle
     wl = _workload(B, C, H, lens, kv_dtype, seed=11)
