@@ -1,20 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of paged absorbed-MLA decode (plan + split scan + combine) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--only]
+                    [--no-side] [--tokens T] [--impl ours|reference]
 
 One step = one pass of the whole hot path over one batch: the split planner, the
 split scan (the dominant kernel) and the LSE combine, on inputs already resident in HBM.
-Prints ONE JSON line on rank 0.  value = KV-read GB/s of the whole job (bytes of cache
-rows the decode must read, summed over ranks, divided by the slowest rank's device
-time); us_per_call is the per-step latency.  The L2 (126 MB) is flushed by a 256 MB
-write between timed steps, outside the timed events.
+Prints ONE JSON line on rank 0.  Its headline workload is long_m256 (B=16, s_q=16,
+H=16, 131,072 cached tokens per request: the largest single-GPU configuration); value =
+KV-read GB/s of the whole job (bytes of cache rows the decode must read, summed over
+ranks, divided by the slowest rank's device time); us_per_call is the per-step latency.
+The L2 (126 MB) is flushed by a 256 MB write between timed steps, outside the timed
+events.  The same run then measures every other workload (tiny, agent_spec,
+ragged_rownorm, fp8_batch) the same way; each has its own record under "workloads",
+with its roofline fraction and its own clock record (--only skips them).
 
 Beside the step the line carries, each timed on its own with CUDA events and the L2
 flushed before every call: the paged KV append of the drafts' rows (kv_append), the
-projections either side of the latent attention (absorb_project), and a long-prefix
-chunked prefill on the same path (prefill: one request, 1024 query tokens x 16 heads at
-the end of a 65,536-token cache).
+projections either side of the latent attention (absorb_project), both per workload,
+and a long-prefix chunked prefill on the same path (prefill: one request, 1024 query
+tokens x 16 heads at the end of a 65,536-token cache).  --tokens T gives every request
+T tokens: a reduced case for profiler captures, never a bench number.
 
 Multi-GPU (torchrun): every rank decodes its own replica of the workload (requests are
 independent; there is no data-path collective), time = max over ranks, scaling weak.
@@ -41,7 +47,7 @@ import numpy as np  # noqa: E402
 
 from mla_attention_decode_paged_b200 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "agent_spec"
+DEFAULT_WORKLOAD = "long_m256"  # the largest single-GPU configuration: B=16, s_q=16, H=16, 131,072 tokens each
 METRIC = "MLA decode \u00b5s/call and KV-read GB/s (% of B200 HBM/tensor roofline)"  # value in GB/s; us_per_call beside it
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # B200 datasheet (dense bf16), for context
@@ -281,25 +287,40 @@ def soak(step, flush_l2, dev, seconds):
         torch.cuda.synchronize(dev)
 
 
-def run_ours(args):
+def roofline_of(wl, scan_avg_s, traffic):
+    """Roofline of the split scan for one launch: HBM-bound (cache bytes) or tensor-bound
+    (2 M T 1088 FLOPs) by the workload's intensity against the measured ridge."""
+    peaks, peak_src = load_peaks()
+    kvb, flops = wl.kv_bytes(), wl.flops()
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / kvb < ridge:
+        roof = {"bound": "hbm", "achieved": kvb / scan_avg_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / scan_avg_s / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe'})"
+    roof["kernel"] = "mla decode split scan"
+    roof["algorithmic_bytes_per_launch"] = kvb
+    roof["algorithmic_flops_per_launch"] = flops
+    nom_peak = NOMINAL_PEAKS["hbm_gbs"] if roof["bound"] == "hbm" else NOMINAL_PEAKS["bf16_tflops"]
+    nominal = {"peak": nom_peak, "unit": roof["unit"], "frac": roof["achieved"] / nom_peak,
+               "note": "B200 datasheet peak, context only"}
+    t_roof = max(kvb / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    return roof, nominal, t_roof
+
+
+def measure_workload(name, args, dev, stream, flush_l2, world, headline):
+    """One workload: the decode step (plan + split scan + combine) timed with CUDA events,
+    the per-kernel pass, clocks sampled during both; for the headline also the CUDA-graph
+    replay and the warm-L2 step; end to end through the public calls with host buffers;
+    and the side paths (KV append, the projections) on the workload's shapes."""
     import torch
-    import torch.distributed as dist
     import mla_attention_decode_paged_b200 as mla
-    from mla_attention_decode_paged_b200 import build as build_mod
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    build_mod.build(quiet=True)
-
-    wl = W.make_workload(args.workload)
+    kw = {} if args.tokens is None else {"seq": ("fixed", args.tokens)}
+    wl = W.make_workload(name, **kw)
     q, kv, bt, sl = (torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).to(dev),
                      (torch.from_numpy(wl.kv.view(np.int16)).view(torch.bfloat16) if wl.kv_dtype == W.KV_BF16
                       else torch.from_numpy(wl.kv)).to(dev),
@@ -307,8 +328,6 @@ def run_ours(args):
     ws = mla.alloc_workspace(wl.B, wl.s_q, wl.H, device=dev)
     out = torch.empty((wl.B, wl.s_q, wl.H, W.DV), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.B, wl.s_q, wl.H), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
         # the three kernels back to back, so that each starts its prologue under the tail
@@ -332,9 +351,6 @@ def run_ours(args):
         mla.combine(ws, wl.B, wl.s_q, wl.H, out, lse, stream=stream)
         ev[3].record(stream)
 
-    def flush_l2(k):
-        flush.fill_(k % 251 + 1)  # a 256 MB write: larger than the 126 MB L2
-
     for _ in range(args.warmup):
         flush_l2(0)
         step()
@@ -342,84 +358,96 @@ def run_ours(args):
     assert mla.device_status(ws, stream=stream) == 0
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     evs_split = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
-        # The timed steps take milliseconds, shorter than the sampler's 200 ms period, so
-        # identical untimed steps run for a soak window before and after them; the clock
-        # record covers the soak and the timed steps together.
+    with ClockSampler(dev.index) as clk:
+        # The timed steps are short next to the sampler's 200 ms period, so identical
+        # untimed steps run for a soak window before and after them; the clock record
+        # covers the soak and the timed steps together.
         soak(step, flush_l2, dev, args.soak_s)
         if world > 1:
-            dist.barrier()
+            torch.distributed.barrier()
         torch.cuda.synchronize(dev)
         for k in range(args.steps):
             flush_l2(k)  # outside the timed events
             step(evs[k])
         torch.cuda.synchronize(dev)
         if world > 1:
-            dist.barrier()
-        # per-kernel pass: the same K steps with events between the kernels
+            torch.distributed.barrier()
         for k in range(args.steps):
             flush_l2(k)
             step_split(evs_split[k])
         torch.cuda.synchronize(dev)
         if world > 1:
-            dist.barrier()
+            torch.distributed.barrier()
         soak(step, flush_l2, dev, args.soak_s)
+    assert mla.device_status(ws, stream=stream) == 0
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     plan_ms = [e[0].elapsed_time(e[1]) for e in evs_split]
     scan_ms = [e[1].elapsed_time(e[2]) for e in evs_split]
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs_split]
     tot_ms, tot_scan_ms = max_over_ranks([sum(step_ms), sum(scan_ms)], world, dev)
+    kvb, flops = wl.kv_bytes(), wl.flops()
+    roof, roof_nominal, t_roof = roofline_of(wl, tot_scan_ms * 1e-3 / args.steps,
+                                             ncu_traffic(name) if args.tokens is None else None)
+    rec = {"workload": workload_desc(wl), "value": job_gbs(kvb, world, args.steps, tot_ms), "unit": "GB/s",
+           "us_per_call": tot_ms / args.steps * 1e3,
+           "tflops": flops * world * args.steps / (tot_ms * 1e-3) / 1e12,
+           "step_us_p10_p50_p90": [float(np.percentile(step_ms, p)) * 1e3 for p in (10, 50, 90)],
+           "breakdown_us": {"plan": statistics.median(plan_ms) * 1e3, "scan": statistics.median(scan_ms) * 1e3,
+                            "combine": statistics.median(comb_ms) * 1e3,
+                            "note": "a second pass of K steps with events between the kernels"},
+           "roofline_us": t_roof * 1e6, "frac_of_roofline_step": t_roof / (tot_ms * 1e-3 / args.steps),
+           "roofline": roof, "roofline_nominal": roof_nominal, "clocks": clk.summary(),
+           "kv_bytes": kvb, "flops": flops}
 
-    # the same step replayed from a CUDA graph (captured once; launch overhead removed)
-    graph = None
-    try:
-        g = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(dev)
-        cap.wait_stream(stream)
-        with torch.cuda.graph(g, stream=cap):
-            mla.plan(sl, wl.s_q, wl.H, ws, stream=cap)
-            mla.decode(q, kv, bt, sl, wl.scale, wl.causal, ws, out, lse, kv_scale=wl.kv_scale, stream=cap)
-        torch.cuda.synchronize(dev)
-        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        for k in range(args.warmup):
-            flush_l2(k)
-            g.replay()
-        torch.cuda.synchronize(dev)
-        for k in range(args.steps):
-            flush_l2(k)
-            gev[k][0].record(stream)
-            g.replay()
-            gev[k][1].record(stream)
-        torch.cuda.synchronize(dev)
-        assert mla.device_status(ws, stream=stream) == 0
-        gms = sorted(e[0].elapsed_time(e[1]) for e in gev)
-        (g_ms,) = max_over_ranks([sum(gms)], world, dev)
-        graph = {"us_per_call": g_ms / args.steps * 1e3, "median_us": statistics.median(gms) * 1e3,
-                 "value": job_gbs(wl.kv_bytes(), world, args.steps, g_ms), "unit": "GB/s"}
-        del g
-    except Exception as e:  # reported, never fatal
-        graph = {"error": f"{type(e).__name__}: {e}"[:200]}
-
-    # the same step with the L2 left warm between steps (no flush): whatever share of the
-    # step's cache rows fits in the L2 can come from it; compared with the L2's size
-    try:
-        wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        for _ in range(args.warmup):
-            step()
-        torch.cuda.synchronize(dev)
-        for k in range(args.steps):
-            step(wev[k])
-        torch.cuda.synchronize(dev)
-        wms = [e[0].elapsed_time(e[1]) for e in wev]
-        (w_ms,) = max_over_ranks([sum(wms)], world, dev)
-        l2_bytes = int(torch.cuda.get_device_properties(dev).L2_cache_size)
-        warm_l2 = {"us_per_call": w_ms / args.steps * 1e3, "median_us": statistics.median(wms) * 1e3,
-                   "value": job_gbs(wl.kv_bytes(), world, args.steps, w_ms), "unit": "GB/s",
-                   "kv_bytes_per_call": wl.kv_bytes(), "l2_bytes": l2_bytes,
-                   "kv_fits_in_l2": wl.kv_bytes() <= l2_bytes,
-                   "note": "same step, no L2 flush between steps; reported beside the flushed numbers, never as them"}
-    except Exception as e:  # reported, never fatal
-        warm_l2 = {"error": f"{type(e).__name__}: {e}"[:200]}
+    if headline:
+        # the same step replayed from a CUDA graph (captured once; launch overhead removed)
+        try:
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap):
+                mla.plan(sl, wl.s_q, wl.H, ws, stream=cap)
+                mla.decode(q, kv, bt, sl, wl.scale, wl.causal, ws, out, lse, kv_scale=wl.kv_scale, stream=cap)
+            torch.cuda.synchronize(dev)
+            gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+            for k in range(args.warmup):
+                flush_l2(k)
+                g.replay()
+            torch.cuda.synchronize(dev)
+            for k in range(args.steps):
+                flush_l2(k)
+                gev[k][0].record(stream)
+                g.replay()
+                gev[k][1].record(stream)
+            torch.cuda.synchronize(dev)
+            assert mla.device_status(ws, stream=stream) == 0
+            gms = sorted(e[0].elapsed_time(e[1]) for e in gev)
+            (g_ms,) = max_over_ranks([sum(gms)], world, dev)
+            rec["graph"] = {"us_per_call": g_ms / args.steps * 1e3, "median_us": statistics.median(gms) * 1e3,
+                            "value": job_gbs(kvb, world, args.steps, g_ms), "unit": "GB/s"}
+            del g
+        except Exception as e:  # reported, never fatal
+            rec["graph"] = {"error": f"{type(e).__name__}: {e}"[:200]}
+        # the same step with the L2 left warm between steps (no flush): whatever share of the
+        # step's cache rows fits in the L2 can come from it; compared with the L2's size
+        try:
+            wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize(dev)
+            for k in range(args.steps):
+                step(wev[k])
+            torch.cuda.synchronize(dev)
+            wms = [e[0].elapsed_time(e[1]) for e in wev]
+            (w_ms,) = max_over_ranks([sum(wms)], world, dev)
+            l2_bytes = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+            rec["warm_l2"] = {"us_per_call": w_ms / args.steps * 1e3, "median_us": statistics.median(wms) * 1e3,
+                              "value": job_gbs(kvb, world, args.steps, w_ms), "unit": "GB/s",
+                              "kv_bytes_per_call": kvb, "l2_bytes": l2_bytes, "kv_fits_in_l2": kvb <= l2_bytes,
+                              "note": "same step, no L2 flush between steps; reported beside the flushed numbers, "
+                                      "never as them"}
+        except Exception as e:  # reported, never fatal
+            rec["warm_l2"] = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     # end to end through the same public calls with host buffers: pinned inputs copied in,
     # outputs copied out, every step.  The cache itself stays resident (it is the state).
@@ -469,126 +497,141 @@ def run_ours(args):
         e2e_step(e2e_ev[k])
     torch.cuda.synchronize(dev)
     (e2e_ms,) = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in e2e_ev)], world, dev)
-    h2d = in_h.numel()
-    d2h = res_h.numel()
-
-    # the write side of the same cache: append the s_q draft rows of each request (rope on
-    # the 64-wide key), timed on its own after everything above (it rewrites those rows)
-    ckv_new = torch.randn((wl.B, wl.s_q, W.DV), device=dev).to(torch.bfloat16)
-    kpe_new = torch.randn((wl.B, wl.s_q, 64), device=dev).to(torch.bfloat16)
-    max_pos = int(wl.seq_lens.max()) + 1
-    ang = torch.arange(max_pos, device=dev, dtype=torch.float64)[:, None] * \
-        (10000.0 ** (-torch.arange(32, device=dev, dtype=torch.float64) / 32.0))[None, :]
-    cos_sin = torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).float().contiguous()
-    app_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for k in range(args.warmup):
-        mla.kv_append(ckv_new, kpe_new, cos_sin, kv, bt, sl, kv_scale=wl.kv_scale, stream=stream)
-    for k in range(args.steps):
-        flush_l2(k)
-        app_ev[k][0].record(stream)
-        mla.kv_append(ckv_new, kpe_new, cos_sin, kv, bt, sl, kv_scale=wl.kv_scale, stream=stream)
-        app_ev[k][1].record(stream)
-    torch.cuda.synchronize(dev)
-    app_us = statistics.median(e[0].elapsed_time(e[1]) for e in app_ev) * 1e3
-    elem = 2 if wl.kv_dtype == W.KV_BF16 else 1
-    app_bytes = wl.B * wl.s_q * (W.DV * 2 + 64 * 2 + 64 * 4 + W.DQK * elem)
-    kv_append_line = {"us_per_call": app_us, "bytes_per_call": app_bytes, "GB/s": app_bytes / (app_us * 1e-6) / 1e9,
-                      "rows": wl.B * wl.s_q, "note": "launch-bound at decode sizes; L2 flushed before each call"}
-
-    # the projections on either side of the latent attention, random weights (no model)
-    q_nope = torch.randn((wl.B, wl.s_q, wl.H, 128), device=dev).to(torch.bfloat16)
-    q_rope = torch.randn((wl.B, wl.s_q, wl.H, 64), device=dev).to(torch.bfloat16)
-    w_uk = (torch.randn((wl.H, W.DV, 128), device=dev) / 128 ** 0.5).to(torch.bfloat16)
-    w_uv = (torch.randn((wl.H, W.DV, 128), device=dev) / W.DV ** 0.5).to(torch.bfloat16)
-    q_abs = torch.empty((wl.B, wl.s_q, wl.H, W.DQK), dtype=torch.bfloat16, device=dev)
-    y_proj = torch.empty((wl.B, wl.s_q, wl.H, 128), dtype=torch.bfloat16, device=dev)
+    rec["e2e"] = {"value": job_gbs(kvb, world, args.steps, e2e_ms), "unit": "GB/s",
+                  "h2d_bytes_per_step": int(in_h.numel()), "d2h_bytes_per_step": int(res_h.numel()),
+                  "us_per_call": e2e_ms / args.steps * 1e3, "device_step_us": tot_ms / args.steps * 1e3,
+                  "note": "q, block_table, seq_lens in (one pinned buffer, one copy) and out, lse back (one copy) "
+                          "per step; the paged cache stays resident"}
 
     def time_op(fn):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
         for _ in range(args.warmup):
             fn()
         for k in range(args.steps):
             flush_l2(k)
-            evs[k][0].record(stream)
+            tev[k][0].record(stream)
             fn()
-            evs[k][1].record(stream)
+            tev[k][1].record(stream)
         torch.cuda.synchronize(dev)
-        return statistics.median(e[0].elapsed_time(e[1]) for e in evs) * 1e3
+        return statistics.median(e[0].elapsed_time(e[1]) for e in tev) * 1e3
 
-    rows = wl.B * wl.s_q * wl.H
-    wbytes = wl.H * W.DV * 128 * 2
-    ab_us = time_op(lambda: mla.absorb_q(q_nope, q_rope, w_uk, q_abs, stream=stream))
-    pj_us = time_op(lambda: mla.project_out(out, w_uv, y_proj, stream=stream))
-    ab_bytes = wbytes + rows * (128 + 64 + W.DQK) * 2
-    pj_bytes = wbytes + rows * (W.DV + 128) * 2
-    absorb_line = {"absorb_q_us": ab_us, "absorb_q_GB/s": ab_bytes / (ab_us * 1e-6) / 1e9,
-                   "project_out_us": pj_us, "project_out_GB/s": pj_bytes / (pj_us * 1e-6) / 1e9,
-                   "weight_bytes_each": wbytes, "note": "per-head W_UK / W_UV [H, 512, 128] bf16, L2 flushed before "
-                                                       "each call; bound by the weights' bytes and launch latency"}
+    if not args.no_side:
+        # the write side of the same cache: append the s_q draft rows of each request (rope on
+        # the 64-wide key), timed on its own after everything above (it rewrites those rows)
+        ckv_new = torch.randn((wl.B, wl.s_q, W.DV), device=dev).to(torch.bfloat16)
+        kpe_new = torch.randn((wl.B, wl.s_q, 64), device=dev).to(torch.bfloat16)
+        max_pos = int(wl.seq_lens.max()) + 1
+        ang = torch.arange(max_pos, device=dev, dtype=torch.float64)[:, None] * \
+            (10000.0 ** (-torch.arange(32, device=dev, dtype=torch.float64) / 32.0))[None, :]
+        cos_sin = torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).float().contiguous()
+        app_us = time_op(lambda: mla.kv_append(ckv_new, kpe_new, cos_sin, kv, bt, sl, kv_scale=wl.kv_scale,
+                                               stream=stream))
+        elem = 2 if wl.kv_dtype == W.KV_BF16 else 1
+        app_bytes = wl.B * wl.s_q * (W.DV * 2 + 64 * 2 + 64 * 4 + W.DQK * elem)
+        rec["kv_append"] = {"us_per_call": app_us, "bytes_per_call": app_bytes,
+                            "GB/s": app_bytes / (app_us * 1e-6) / 1e9, "rows": wl.B * wl.s_q,
+                            "note": "launch-bound at decode sizes; L2 flushed before each call"}
+        # the projections on either side of the latent attention, random weights (no model)
+        q_nope = torch.randn((wl.B, wl.s_q, wl.H, 128), device=dev).to(torch.bfloat16)
+        q_rope = torch.randn((wl.B, wl.s_q, wl.H, 64), device=dev).to(torch.bfloat16)
+        w_uk = (torch.randn((wl.H, W.DV, 128), device=dev) / 128 ** 0.5).to(torch.bfloat16)
+        w_uv = (torch.randn((wl.H, W.DV, 128), device=dev) / W.DV ** 0.5).to(torch.bfloat16)
+        q_abs = torch.empty((wl.B, wl.s_q, wl.H, W.DQK), dtype=torch.bfloat16, device=dev)
+        y_proj = torch.empty((wl.B, wl.s_q, wl.H, 128), dtype=torch.bfloat16, device=dev)
+        rows = wl.B * wl.s_q * wl.H
+        wbytes = wl.H * W.DV * 128 * 2
+        ab_us = time_op(lambda: mla.absorb_q(q_nope, q_rope, w_uk, q_abs, stream=stream))
+        pj_us = time_op(lambda: mla.project_out(out, w_uv, y_proj, stream=stream))
+        ab_bytes = wbytes + rows * (128 + 64 + W.DQK) * 2
+        pj_bytes = wbytes + rows * (W.DV + 128) * 2
+        proj_flops = 2 * rows * W.DV * 128
+        rec["absorb_project"] = {"absorb_q_us": ab_us, "absorb_q_GB/s": ab_bytes / (ab_us * 1e-6) / 1e9,
+                                 "project_out_us": pj_us, "project_out_GB/s": pj_bytes / (pj_us * 1e-6) / 1e9,
+                                 "flops_each": proj_flops, "absorb_q_tflops": proj_flops / (ab_us * 1e-6) / 1e12,
+                                 "project_out_tflops": proj_flops / (pj_us * 1e-6) / 1e12,
+                                 "weight_bytes_each": wbytes,
+                                 "note": "per-head W_UK / W_UV [H, 512, 128] bf16, L2 flushed before each call"}
+    del q, kv, bt, sl, ws, out, lse, in_d, res_d
+    torch.cuda.empty_cache()
+    return wl, rec
 
-    try:
-        prefill_line = prefill_measure(args, dev, stream, flush_l2, time_op)
-    except (RuntimeError, mla.MlaError) as e:  # reported in the line; the decode numbers stand
-        prefill_line = {"error": str(e)}
 
-    kvb = wl.kv_bytes()
-    flops = wl.flops()
-    value = job_gbs(kvb, world, args.steps, tot_ms)
-    e2e_value = job_gbs(kvb, world, args.steps, e2e_ms)
-    peaks, peak_src = load_peaks()
-    scan_avg_s = tot_scan_ms * 1e-3 / args.steps
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    intensity = flops / kvb
-    if intensity < ridge:
-        roof = {"bound": "hbm", "achieved": kvb / scan_avg_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": flops / scan_avg_s / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    nom_peak = NOMINAL_PEAKS["hbm_gbs"] if roof["bound"] == "hbm" else NOMINAL_PEAKS["bf16_tflops"]
-    roof_nominal = {"peak": nom_peak, "unit": roof["unit"], "frac": roof["achieved"] / nom_peak,
-                    "note": "B200 datasheet peak, context only"}
-    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe'})"
-    roof["kernel"] = "mla decode split scan"
-    roof["traffic"] = ncu_traffic(args.workload)
-    roof["algorithmic_bytes_per_launch"] = kvb
-    roof["algorithmic_flops_per_launch"] = flops
-    t_roof = max(kvb / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mla_attention_decode_paged_b200 as mla
+    from mla_attention_decode_paged_b200 import build as build_mod
 
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "us_per_call": tot_ms / args.steps * 1e3,
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    build_mod.build(quiet=True)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush_l2(k):
+        flush.fill_(k % 251 + 1)  # a 256 MB write: larger than the 126 MB L2
+
+    names = [args.workload] + ([] if args.only else [n for n in W.WORKLOAD_ORDER if n != args.workload])
+    recs = {}
+    head_wl = None
+    for n in names:
+        wl, rec = measure_workload(n, args, dev, stream, flush_l2, world, headline=(n == args.workload))
+        recs[n] = rec
+        if n == args.workload:
+            head_wl = wl
+    head = recs[args.workload]
+
+    def time_op(fn):
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for _ in range(args.warmup):
+            fn()
+        for k in range(args.steps):
+            flush_l2(k)
+            tev[k][0].record(stream)
+            fn()
+            tev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.median(e[0].elapsed_time(e[1]) for e in tev) * 1e3
+
+    prefill_line = None
+    if not args.no_side:
+        try:
+            prefill_line = prefill_measure(args, dev, stream, flush_l2, time_op)
+        except (RuntimeError, mla.MlaError) as e:  # reported in the line; the decode numbers stand
+            prefill_line = {"error": str(e)}
+
+    wl = head_wl
+    line = {"metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["us_per_call"] * 1e-3, "us_per_call": head["us_per_call"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.kv_dtype == W.KV_BF16 else "e4m3->bf16",
             "data": "synthetic (seeded N(0,1) q/KV; no dataset)",
-            "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": int(wl.seq_lens.max()),
+            "config": {"workload": head["workload"], "global_batch": wl.B * world, "seq_len": int(wl.seq_lens.max()),
                        "parallelism": f"replicas x{world} (no collective)",
                        "l2": "flushed between steps by a 256 MB write outside the timed events"},
-            "breakdown_us": {"plan": statistics.median(plan_ms) * 1e3, "scan": statistics.median(scan_ms) * 1e3,
-                             "combine": statistics.median(comb_ms) * 1e3,
-                             "note": "a second pass of K steps with events between the kernels"},
-            "tflops": flops * world * args.steps / (tot_ms * 1e-3) / 1e12,
-            "roofline_us": t_roof * 1e6, "frac_of_roofline_step": t_roof / (tot_ms * 1e-3 / args.steps),
-            "roofline": roof,
-            "roofline_nominal": roof_nominal,
-            "step_us_p10_p50_p90": [float(np.percentile(step_ms, 10)) * 1e3, float(np.percentile(step_ms, 50)) * 1e3,
-                                    float(np.percentile(step_ms, 90)) * 1e3],
-            "graph": graph,
-            "warm_l2": warm_l2,
-            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "us_per_call": e2e_ms / args.steps * 1e3,
-                    "note": "q, block_table, seq_lens in (one pinned buffer, one copy) and out, lse back (one copy) "
-                            "per step; the paged cache stays resident"},
-            "kv_append": kv_append_line,
-            "absorb_project": absorb_line,
+            "breakdown_us": head["breakdown_us"], "tflops": head["tflops"],
+            "roofline_us": head["roofline_us"], "frac_of_roofline_step": head["frac_of_roofline_step"],
+            "roofline": head["roofline"], "roofline_nominal": head["roofline_nominal"],
+            "step_us_p10_p50_p90": head["step_us_p10_p50_p90"],
+            "graph": head.get("graph"), "warm_l2": head.get("warm_l2"), "e2e": head["e2e"],
+            "kv_append": head.get("kv_append"), "absorb_project": head.get("absorb_project"),
             "prefill": prefill_line,
+            "workloads": {n: {k: v for k, v in r.items() if k not in ("graph", "warm_l2")} for n, r in recs.items()},
             "gpu_launches": 3 * args.steps,
-            "gpu_launches_per_kernel_pass": 3 * args.steps,
-            "gpu_launches_graph_pass": 3 * args.steps,
-            "clocks": clk.summary()}
+            "gpu_launches_note": "plan + split scan + combine per timed step of the headline workload",
+            "clocks": head["clocks"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         full_s, cores, desc = oracle_baseline(wl)
-        line["cpu_baseline"] = {"value": kvb / full_s / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": desc}
+        line["cpu_baseline"] = {"value": wl.kv_bytes() / full_s / 1e9, "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -605,6 +648,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soak-s", type=float, default=1.0, help="untimed identical steps around the timed ones")
+    ap.add_argument("--only", action="store_true", help="measure the headline workload alone")
+    ap.add_argument("--no-side", action="store_true", help="skip the KV append, projection and prefill timings")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="every request this many tokens (a reduced case for profiler captures; the line's "
+                         "config says so)")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warmup raised to 3 (minimum)")

@@ -258,8 +258,11 @@ mla_status mla_get_device_status(void* workspace, int* code, void* stream);
  * MLA_ERR_WORKSPACE_TOO_SMALL (use mla_decode with your own workspace instead); the
  * five reference workloads, up to B = 32 requests of s_q * H = 256 rows, fit.
  *
- * The first call on a device looks up the scratch array's device address (with that
- * device current) and caches it; make that first call before any stream capture.
+ * Every call made outside stream capture looks up the scratch array's device address on
+ * the current device (cudaGetSymbolAddress, which allocates nothing), so a device reset
+ * that reloads the library's module is harmless; a call made while `stream` is being
+ * captured uses the address found by the last uncaptured call on that device instead,
+ * so make one uncaptured call first (and again after a device reset).
  * Every call shares the one array and the array keeps the last call's contents: the
  * planner rewrites everything that a call reads before reading it, but calls whose
  * work overlaps on the GPU (several streams, or several host threads on one device)

@@ -75,18 +75,27 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     // L = log2 sum_j 2^lse2_j per row: warp w < 8 takes rows 2w and 2w + 1 (one per half-warp)
     if (tid < kTileThreads) {
         const int lane = tid & 31, r = 2 * (tid >> 5) + (lane >> 4), k = lane & 15;
+        // fmaxf drops NaN, so a poisoned split (NaN lse2: a bad page or length) is tracked
+        // on its own and turns the merged row into NaN even when every split is poisoned
         float mx = -INFINITY;
-        for (int j = k; j < ns; j += 16) mx = fmaxf(mx, lbase[j * lstride + r]);
+        bool poisoned = false;
+        for (int j = k; j < ns; j += 16) {
+            const float l2 = lbase[j * lstride + r];
+            poisoned |= l2 != l2;
+            mx = fmaxf(mx, l2);
+        }
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        poisoned = ((__ballot_sync(0xffffffffu, poisoned) >> (lane & 16)) & 0xffffu) != 0;  // this row's half-warp
         float sum = 0.f;
         if (mx != -INFINITY)
             for (int j = k; j < ns; j += 16) sum += fast_exp2(lbase[j * lstride + r] - mx);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (k == 0) {
-            Lsh[r] = mx + __log2f(sum);
-            Msh[r] = mx;
+            const float nanv = __int_as_float(0x7fc00000);
+            Lsh[r] = poisoned ? nanv : mx + __log2f(sum);
+            Msh[r] = poisoned ? nanv : mx;
         }
     }
     __syncthreads();

@@ -9,8 +9,8 @@
 // which every GPU that loads the library holds until the process exits.
 //
 // In host code the array's name is only a host-side stand-in, never a device address,
-// so the device address is looked up once per device with cudaGetSymbolAddress (with
-// that device current) and passed to the kernels like any workspace pointer.
+// so its device address is looked up with cudaGetSymbolAddress (with the caller's device
+// current) and passed to the kernels like any workspace pointer.
 #include <mutex>
 
 #include "mla_decode_params.cuh"
@@ -25,12 +25,18 @@ static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxCachedDevices] = {};
 
-// Device address of g_scratch on the current device (looked up on first use per device).
-mla_status scratch_address(void** out) {
+// Device address of g_scratch on the current device.  Outside stream capture it is looked
+// up on every call (cudaGetSymbolAddress allocates nothing), so a context that was reset
+// and reloaded the module never gets a stale address.  Inside a capture the lookup is not
+// made; the address cached by the last call outside capture is used instead.
+mla_status scratch_address(cudaStream_t stream, void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MLA_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MLA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (dev < kMaxCachedDevices && g_scratch_addr[dev] != nullptr) {
+    if (cap != cudaStreamCaptureStatusNone) {
+        if (dev >= kMaxCachedDevices || g_scratch_addr[dev] == nullptr) return MLA_ERR_CUDA;
         *out = g_scratch_addr[dev];
         return MLA_OK;
     }
@@ -55,7 +61,7 @@ extern "C" mla_status mla_decode_noalloc(const void* q, const void* kv_pages, in
     const mla::WsLayout L = mla::make_layout(B, s_q, H, mla::num_groups_for(sms, mla::num_row_blocks(s_q, H)));
     if ((size_t)L.total > kScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
     void* ws = nullptr;
-    mla_status st = scratch_address(&ws);
+    mla_status st = scratch_address((cudaStream_t)stream, &ws);
     if (st != MLA_OK) return st;
     // The plan rewrites the whole header, the status word included, so nothing left in
     // the scratch by an earlier call is read before it is written again.

@@ -130,7 +130,7 @@ __device__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 __device__ __forceinline__ bool request_ok(const DecodeParams& p, int T) {
-    return T >= 1 && T <= p.max_pages * kPage && !(p.causal && T < p.s_q);
+    return T >= 1 && (int64_t)T <= (int64_t)p.max_pages * kPage && !(p.causal && T < p.s_q);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -721,21 +721,59 @@ int sm100_cta_slots() {
     return n;
 }
 
+// The tensor map of the cache depends only on (device, cache pointer, page count); a
+// decode step calls the scan once per layer with the same few caches, so the last map
+// each host thread encoded is kept and reused while those match.
+struct TmapCacheEntry {
+    int dev = -1;
+    const void* kv = nullptr;
+    int64_t num_pages = -1;
+    CUtensorMap map;
+};
+
+template <int KV>
+bool cached_kv_map(int dev, const DecodeParams& p, CUtensorMap* out) {
+    static thread_local TmapCacheEntry e;
+    if (e.dev != dev || e.kv != p.kv || e.num_pages != p.num_pages) {
+        const uint64_t kvrows = (uint64_t)p.num_pages * kPage;
+        const bool ok = KV == MLA_KV_E4M3
+                            ? make_map_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.kv, kDqk, kvrows, kDqk, 64, kTok,
+                                          CU_TENSOR_MAP_SWIZZLE_NONE)
+                            : make_map_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 64,
+                                          kTok, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok) {
+            e.dev = -1;
+            return false;
+        }
+        e.dev = dev;
+        e.kv = p.kv;
+        e.num_pages = p.num_pages;
+    }
+    *out = e.map;
+    return true;
+}
+
+// The dynamic shared memory opt-in is a per-device property of the kernel: set once.
+template <int KV>
+bool smem_attribute_set(int dev) {
+    static int done[64] = {};
+    if (dev < 64 && done[dev]) return true;
+    if (cudaFuncSetAttribute(decode_sm100_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+        cudaSuccess)
+        return false;
+    if (dev < 64) done[dev] = 1;
+    return true;
+}
+
 template <int KV>
 mla_status launch_typed(const DecodeParams& p, cudaStream_t stream) {
     Sm100Args a;
     memset(&a, 0, sizeof(a));
     a.p = p;
-    const uint64_t kvrows = (uint64_t)p.num_pages * kPage;
-    const bool ok = KV == MLA_KV_E4M3
-                        ? make_map_2d(&a.tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.kv, kDqk, kvrows, kDqk, 64, kTok,
-                                      CU_TENSOR_MAP_SWIZZLE_NONE)
-                        : make_map_2d(&a.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 64,
-                                      kTok, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok) return MLA_ERR_CUDA;
-    if (cudaFuncSetAttribute(decode_sm100_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
-        return MLA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (!cached_kv_map<KV>(dev, p, &a.tm_kv)) return MLA_ERR_CUDA;
+    if (!smem_attribute_set<KV>(dev)) return MLA_ERR_CUDA;
     const int ctas = p.groups_launched * num_row_blocks(p.s_q, p.H);
     // programmatic dependent launch: the prologue (barriers, TMEM, tensor map) overlaps the
     // tail of the previous grid in the stream; the kernel waits for it before any global access

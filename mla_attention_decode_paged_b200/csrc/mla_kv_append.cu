@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(32 * kAppendWarps) kv_append_kernel(
     const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(kpe + r * 64)[lane];
     const int T = seq_lens[b];
     const int pos = T - s_q + i;
-    bool ok = T >= s_q && T <= max_pages * kPage && pos < max_pos;
+    bool ok = T >= s_q && (int64_t)T <= (int64_t)max_pages * kPage && pos < max_pos;
     int32_t page = -1;
     float cj = 0.f, sj = 0.f;
     if (ok) {

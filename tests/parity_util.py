@@ -51,8 +51,9 @@ def to_device(wl, device="cuda"):
     return q, kv, bt, sl
 
 
-def run_gpu(wl, num_sms: int = 0, device="cuda", tensors=None, check_status=True):
-    """Plan + decode on the GPU; returns (out float32 numpy, lse numpy)."""
+def run_gpu(wl, num_sms: int = 0, device="cuda", tensors=None, check_status=True, return_ws=False):
+    """Plan + decode on the GPU; returns (out float32 numpy, lse numpy), and the workspace
+    tensor (which holds the plan) when ``return_ws``."""
     import torch
     import mla_attention_decode_paged_b200 as mla
     q, kv, bt, sl = tensors if tensors is not None else to_device(wl, device)
@@ -65,7 +66,22 @@ def run_gpu(wl, num_sms: int = 0, device="cuda", tensors=None, check_status=True
     if check_status:
         code = mla.device_status(ws)
         assert code == 0, f"device status {code}"
+    if return_ws:
+        return out.float().cpu().numpy(), lse.cpu().numpy(), ws
     return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def read_plan(ws):
+    """The plan in a workspace, read back to the host: (header int32 words, group -> first
+    segment, request -> first segment, segments [n, 4] = (b, first page, end page, split))."""
+    raw = ws.cpu().numpy()
+    h32 = raw[:48].view(np.int32)
+    h64 = raw[48:96].view(np.int64)
+    G, nseg, B = int(h32[7]), int(h32[8]), int(h32[3])
+    gb = raw[h64[0]:h64[0] + 4 * (G + 1)].view(np.int32)
+    rs = raw[h64[1]:h64[1] + 4 * (B + 1)].view(np.int32)
+    segs = raw[h64[2]:h64[2] + 16 * nseg].view(np.int32).reshape(-1, 4)
+    return h32, gb, rs, segs
 
 
 def run_oracle(wl, heads=None, requests=None):

@@ -1,8 +1,9 @@
 """GPU parity of libmla_decode.so against the float64 oracle, through the C ABI.
 
 Small cases compare every output element; the full-size workloads run in the same
-launch configuration as bench.py and compare sampled rows (the first and last request,
-the first and last head, every draft token) that the oracle computes one by one.
+launch configuration as bench.py and compare sampled rows that the oracle computes one
+by one (a request the plan split and one it held whole where the workload has both,
+seeded heads, every draft token); a planted key checks the draft mask at full length.
 Every workload carries NaN canaries in page tails and spare pages.
 """
 import numpy as np
@@ -104,18 +105,6 @@ def test_page_permutation_leaves_the_result_within_rounding():
     assert np.abs(out1 - out2).max() < 2e-2
 
 
-def _read_plan(ws):
-    import torch
-    raw = ws.cpu().numpy()
-    h32 = raw[:48].view(np.int32)
-    h64 = raw[48:96].view(np.int64)
-    G, nseg, B = int(h32[7]), int(h32[8]), int(h32[3])
-    gb = raw[h64[0]:h64[0] + 4 * (G + 1)].view(np.int32)
-    rs = raw[h64[1]:h64[1] + 4 * (B + 1)].view(np.int32)
-    segs = raw[h64[2]:h64[2] + 16 * nseg].view(np.int32).reshape(-1, 4)
-    return h32, gb, rs, segs
-
-
 @pytest.mark.parametrize("lens,s_q,H,num_sms", [([65536] * 4, 4, 16, 148), ([70000, 1, 64, 65, 30000], 2, 128, 148),
                                                 ([300] * 3, 8, 32, 8), ([5] * 7, 1, 16, 1),
                                                 (list(np.random.default_rng(1).integers(1, 3000, 600)), 1, 16, 148),
@@ -127,7 +116,7 @@ def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     ws = mla.alloc_workspace(len(lens), s_q, H, num_sms=num_sms)
     mla.plan(sl, s_q, H, ws, num_sms=num_sms)
     torch.cuda.synchronize()
-    h32, gb, rs, segs = _read_plan(ws)
+    h32, gb, rs, segs = pu.read_plan(ws)
     G = plan_ref.num_groups_for(num_sms, (s_q * H + 63) // 64)
     egb, ers, esegs = plan_ref.plan(lens, G)
     assert h32[2] == 0x4D4C4131 and h32[7] == G
@@ -149,6 +138,8 @@ def test_bad_page_id_sets_device_status_and_poisons_only_that_request():
     assert mla.device_status(ws) == 0  # cleared by the read
     o = out.float().cpu().numpy()
     assert np.all(np.isnan(o[1])) and np.all(np.isfinite(o[0])) and np.all(np.isfinite(o[2]))
+    l = lse.cpu().numpy()
+    assert np.all(np.isnan(l[1])) and np.all(np.isfinite(l[[0, 2]]))
 
 
 def test_seq_len_beyond_block_table_sets_device_status():
@@ -164,20 +155,95 @@ def test_seq_len_beyond_block_table_sets_device_status():
     mla.decode(q, kv, bt, sl_bad, wl.scale, True, ws, out, lse)
     assert mla.device_status(ws) == 5
     assert np.all(np.isnan(out[1].float().cpu().numpy()))
+    assert np.all(np.isnan(lse[1].cpu().numpy())), "a poisoned split request reports NaN lse too"
+    assert np.all(np.isfinite(lse[0].cpu().numpy()))
+
+
+def _sample_requests_and_heads(wl, segs, seed):
+    """Requests the plan split and requests it held whole (the first of each, where the
+    workload has them), one more seeded request, and heads {0, H-1} plus three seeded
+    heads."""
+    rng = np.random.default_rng(seed)
+    split = sorted({int(b) for b, _, _, sp in segs if sp})
+    whole = sorted({int(b) for b, _, _, sp in segs if not sp})
+    reqs = {split[0]} if split else set()
+    if whole:
+        reqs.add(whole[0])
+    reqs.add(int(rng.integers(0, wl.B)))
+    heads = {0, wl.H - 1} | {int(h) for h in rng.choice(wl.H, size=min(3, wl.H), replace=False)}
+    return sorted(reqs), sorted(heads), split, whole
 
 
 @pytest.mark.parametrize("name", ["agent_spec", "ragged_rownorm", "long_m256", "fp8_batch"])
 def test_full_size_workload_sampled_rows(name):
-    """The full workload in the bench's launch configuration; oracle on sampled rows."""
+    """The full workload in the bench's launch configuration; the oracle on sampled rows of a
+    request the plan split (partials + combine) and of one it held whole (direct bf16 out),
+    where the workload has both, on seeded heads and every draft token."""
     wl = W.make_workload(name)
-    out, lse = pu.run_gpu(wl)
-    reqs = [0, wl.B - 1]
-    heads = [0, wl.H - 1]
+    out, lse, ws = pu.run_gpu(wl, return_ws=True)
+    _, _, _, segs = pu.read_plan(ws)
+    reqs, heads, split, whole = _sample_requests_and_heads(wl, segs, seed=W.WORKLOAD_ORDER.index(name))
+    assert split, "the bench configuration splits at least one request"
+    if name == "fp8_batch":
+        assert whole, "the ragged fp8 batch has requests that one share holds whole"
+        assert any(b in whole for b in reqs) and any(b in split for b in reqs)
     ref_out, ref_lse = pu.run_oracle(wl, heads=heads, requests=reqs)
     got_out = out[reqs][:, :, heads]
     got_lse = lse[reqs][:, :, heads]
-    pu.check_close(got_out, got_lse, ref_out, ref_lse, wl.kv_dtype, what=name)
+    pu.check_close(got_out, got_lse, ref_out, ref_lse, wl.kv_dtype, what=f"{name} requests {reqs} heads {heads}")
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+
+
+def _plant(wl, b, h0):
+    """A cache row at position T_b - 1 of request b whose score with draft s_q - 1, head h0
+    is huge: every value is +-the largest magnitude, with the sign of that query."""
+    T = int(wl.seq_lens[b])
+    page, slot = int(wl.block_table[b, (T - 1) // 64]), (T - 1) % 64
+    sign = np.sign(W.bf16_bits_to_float32(wl.q[b, wl.s_q - 1, h0]))
+    if wl.kv_dtype == W.KV_BF16:
+        row = W._bf16_bits(np.where(sign >= 0, 8.0, -8.0).astype(np.float32))
+    else:
+        row = np.where(sign >= 0, 0x7E, 0xFE).astype(np.uint8)  # e4m3 +-448
+    return page, slot, row
+
+
+@pytest.mark.parametrize("name", ["agent_spec", "fp8_batch"])
+def test_planted_key_at_full_length_reaches_only_the_last_draft(name):
+    """At full length a mask error moves an output far less than the tolerance, so the mask
+    is checked with a planted key: a huge-score row at position T_b - 1 (visible to draft
+    s_q - 1 only).  Every other row of the batch must come out bit-identical to the run
+    without it, and the last draft's row must snap to the planted row, as in the oracle."""
+    import torch
+    import mla_attention_decode_paged_b200 as mla
+    wl = W.make_workload(name)
+    b = int(np.argmax(wl.seq_lens)) if name == "fp8_batch" else 1
+    h0 = 3
+    tensors = pu.to_device(wl)
+    base_out, base_lse, ws = pu.run_gpu(wl, tensors=tensors, return_ws=True)
+    _, _, rs, _ = pu.read_plan(ws)
+    assert rs[b + 1] - rs[b] > 1, "the planted request is split over several CTAs"
+    page, slot, row = _plant(wl, b, h0)
+    kv = tensors[1]
+    row_t = torch.from_numpy(row.view(np.int16) if wl.kv_dtype == W.KV_BF16 else row)
+    if wl.kv_dtype == W.KV_BF16:
+        row_t = row_t.view(torch.bfloat16)
+    kv[page, slot] = row_t.to(kv.device)
+    out, lse = pu.run_gpu(wl, tensors=tensors)
+    last = wl.s_q - 1
+    keep = np.ones(out.shape[:3], dtype=bool)
+    keep[b, last] = False
+    assert np.array_equal(out[keep], base_out[keep]), "a row that cannot see the planted key changed"
+    assert np.array_equal(lse[keep], base_lse[keep]), "an lse that cannot see the planted key changed"
+    # the last draft of request b against the oracle on the planted cache
+    wl.kv[page, slot] = row
+    heads = [0, h0, wl.H - 1]
+    ref_out, ref_lse = pu.run_oracle(wl, heads=heads, requests=[b])
+    pu.check_close(out[[b]][:, :, heads], lse[[b]][:, :, heads], ref_out, ref_lse, wl.kv_dtype, what="planted")
+    planted = (W.bf16_bits_to_float32(row) if wl.kv_dtype == W.KV_BF16 else
+               np.where(row == 0x7E, 448.0, -448.0) * wl.kv_scale)[:512]
+    np.testing.assert_allclose(out[b, last, h0], planted, rtol=2e-2, atol=2e-2)
+    # and the earlier drafts of request b stay far from it
+    assert np.abs(out[b, :last, h0] - planted).min() > 1.0
 
 
 def test_bounded_wait_gives_up_with_a_status_and_the_context_stays_usable():

@@ -3,9 +3,10 @@
 cudaMalloc's implicit synchronisation).  It runs on the library's static scratch array
 instead of a caller workspace.
 
-Checked through the C ABI against mla_decode with a caller workspace, within the
-parity tolerances, on two calls in a row (the second call finds the first call's
-leftovers in the shared scratch).  This file is collected last on purpose.
+Checked through the C ABI, on two calls in a row (the second call finds the first
+call's leftovers in the shared scratch), against the float64 oracle and against
+mla_decode with a caller workspace, within the parity tolerances.  This file is
+collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -37,17 +38,19 @@ def _noalloc(wl, tensors, out, lse):
 
 @pytest.mark.parametrize("name,kw", [("agent_spec", dict(B=3, seq=("fixed", 2000))),
                                      ("fp8_batch", dict(B=4, seq=("lognormal", 500, 1.0, 65, 3000)))])
-def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(name, kw):
+def test_noalloc_matches_the_oracle_and_the_workspace_entry_point_on_two_calls_in_a_row(name, kw):
     import torch
     wl = W.make_workload(name, **kw)
     tensors = pu.to_device(wl)
-    ref_out, ref_lse = pu.run_gpu(wl, tensors=tensors)
+    ws_out, ws_lse = pu.run_gpu(wl, tensors=tensors)
+    ref_out, ref_lse = pu.run_oracle(wl)
     for call in range(2):
         out = torch.full((wl.B, wl.s_q, wl.H, W.DV), float("nan"), dtype=torch.bfloat16, device="cuda")
         lse = torch.full((wl.B, wl.s_q, wl.H), float("nan"), dtype=torch.float32, device="cuda")
         got_out, got_lse = _noalloc(wl, tensors, out, lse)
-        pu.check_close(got_out, got_lse, ref_out.astype(np.float64), ref_lse.astype(np.float64), wl.kv_dtype,
-                       what=f"noalloc call {call}")
+        pu.check_close(got_out, got_lse, ref_out, ref_lse, wl.kv_dtype, what=f"noalloc call {call} vs the oracle")
+        pu.check_close(got_out, got_lse, ws_out.astype(np.float64), ws_lse.astype(np.float64), wl.kv_dtype,
+                       what=f"noalloc call {call} vs mla_decode")
 
 
 def test_noalloc_rejects_a_shape_beyond_its_scratch():
