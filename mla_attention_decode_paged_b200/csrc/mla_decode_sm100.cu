@@ -10,22 +10,36 @@
 // Tensor memory (128 lanes x 512 columns) with 64-row MMAs, whose rows occupy 16 lanes
 // of each 32-lane subpartition:
 //   lanes at offset 0  : O, the 64 x 512 fp32 output accumulator (all 512 columns)
-//   lanes at offset 16 : q (64 x 576 bf16, 288 columns, loaded once per split) and two
+//   lanes at offset 16 : q (loaded once per split: 64 x 576 bf16, or for an e4m3 cache
+//                        two e4m3 terms of 64 x 576; 288 columns either way) and two
 //                        64-column score buffers.
-// Per page:
+// Per page, bf16 cache (kind::f16 MMAs):
 //   TMA (producer warp): the page's 64 rows x 576 columns as nine 64-column boxes with
-//       128-byte swizzle (one 72 KB stage; three stages).  An e4m3 page lands as nine
-//       unswizzled 64 x 64-byte boxes in the upper half of each bf16 slot, and four more
-//       warps widen it to bf16 in place (exact); kv_scale is folded into the score and
-//       output scales.
-//   MMA (one thread): S = q . K^T with q read from TMEM (M=64 N=64, 36 K-steps), then
-//       O += P . V with P (bf16) and V (the same page, read MN-major) from shared memory
-//       (M=64 N=256, twice, 4 K-steps each).  P is written over the page's rope chunk,
-//       which only the score MMAs read: every stage carries its own P, and the softmax
-//       of a page never waits for the previous page's PV.
+//       128-byte swizzle (one 72 KB stage; three stages).
+//   MMA (one thread): S = q . K^T with q read from TMEM (M=64 N=64 K=16, 36 K-steps),
+//       then O += P . V with P (bf16) and V (the same page, read MN-major) from shared
+//       memory (M=64 N=256 K=16, twice, 4 K-steps each).
+// Per page, e4m3 cache (kind::f8f6f4 MMAs, both operands e4m3: the cache bytes are read
+//   by the tensor cores as they are, with kv_scale folded into the score and output
+//   scales):
+//   TMA: nine 64 x 64-byte boxes with 64-byte swizzle (one 36 KB stage; six stages).
+//   MMA: S = (q_hi + q_lo) . K^T, two chains of 18 K-steps (M=64 N=64 K=32) into one
+//       accumulator, where per row q_hi = e4m3(q / s_r), q_lo = e4m3(q / s_r - q_hi) and
+//       s_r is the smallest power of two with max|q_r| / s_r <= 448: q / s_r is then still
+//       a bf16 value, whose 8 significant bits the two 4-bit terms hold exactly (bar
+//       e4m3's subnormal range), so the scores are those of the bf16 q.  Then
+//       O += (P_hi + P_lo) . V with P_hi = e4m3(P), P_lo = e4m3(P - P_hi) (M=64 N=256 K=32:
+//       2 terms x 2 halves x 2 K-steps), P to 8 significant bits as a bf16 P would be.
+//       One e4m3 term of q moves lse past 1e-3, and one of P moves short rows past the
+//       relative L2 bound.
+// Either way P is written over the page's rope chunk (the e4m3 P_lo into a two-entry
+// ring), which only the score MMAs read: every stage carries its own P, and the softmax
+// of a page never waits for the previous page's PV.
 //   softmax (4 warps, 16 rows each, two threads per row with 32 scores each): base-2
 //       online softmax with the causal draft mask; the running max is only raised (and
-//       O rescaled) when a score exceeds it by more than 8, so P <= 256.
+//       O rescaled) when a score exceeds it by more than 8 (bf16) or 4 (e4m3), and the
+//       e4m3 P is 2^(x - m + 4): P <= 256 < 448, with the bulk of a long near-uniform row
+//       far above e4m3's subnormal floor.
 //   epilogue: O / l -> bf16 out (a request the split holds whole) or an fp32 partial and
 //       its base-2 lse (split request; merged by the combine kernel).
 #include <cudaTypedefs.h>
@@ -42,32 +56,54 @@ namespace {
 
 constexpr int kRows = kRowsPerBlock;  // 64 folded rows per CTA (MMA M)
 constexpr int kTok = 64;              // tokens per page (S MMA N)
-constexpr int kStages = 3;
-// warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue, and for an e4m3 cache warps 6-9
-// widen each landed page to bf16 in place
-constexpr int kThreadsBf16 = 192;
-constexpr int kThreadsE4m3 = 320;
-template <int KV>
-constexpr int threads_for() { return KV == MLA_KV_E4M3 ? kThreadsE4m3 : kThreadsBf16; }
+// warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue
+constexpr int kThreads = 192;
 static_assert(kRows == 64, "the TMEM layout below is the 64-row MMA layout");
 
-constexpr uint32_t kChunk = kTok * 128;              // 64 tokens x 64 columns bf16, 128B-swizzled
-constexpr uint32_t kStageBytes = 9 * kChunk;         // 8 latent chunks + 1 rope chunk: 72 KB
-constexpr uint32_t kRawChunk = kTok * 64;            // e4m3: 64 tokens x 64 columns, in the upper half
-constexpr uint32_t kRawStageBytes = 9 * kRawChunk;   //        of each bf16 chunk slot
+// Shared-memory geometry per cache type.  A chunk is 64 tokens x 64 columns of one page,
+// 8-row swizzle atoms; a stage holds one page (8 latent chunks + the rope chunk).
+template <int KV>
+struct Geo;
+template <>
+struct Geo<MLA_KV_BF16> {
+    static constexpr int kStages = 3;
+    static constexpr uint32_t kChunk = kTok * 128;   // 128-byte rows, 128-byte swizzle
+    static constexpr uint32_t kSbo = 8 * 128;
+    static constexpr uint32_t kSwizzle = ptx::kSwizzle128;
+    static constexpr float kRescale = 8.f;           // raise the running max past this margin
+    static constexpr float kPOffset = 0.f;           // P = 2^(x - m + offset)
+};
+template <>
+struct Geo<MLA_KV_E4M3> {
+    static constexpr int kStages = 6;
+    static constexpr uint32_t kChunk = kTok * 64;    // 64-byte rows, 64-byte swizzle
+    static constexpr uint32_t kSbo = 8 * 64;
+    static constexpr uint32_t kSwizzle = ptx::kSwizzle64;
+    static constexpr float kRescale = 4.f;
+    static constexpr float kPOffset = 4.f;
+};
+constexpr int kMaxStages = 6;
+template <int KV>
+constexpr uint32_t stage_bytes() { return 9 * Geo<KV>::kChunk; }
+
 constexpr uint32_t kOffKv = 0;
-constexpr uint32_t kOffPInStage = 8 * kChunk;        // P (64 rows x 64 tokens bf16) over the rope chunk
-constexpr uint32_t kOffEpi = kOffKv + kStages * kStageBytes;  // epilogue staging: 2 KB per softmax warp
+// after the stages (221,184 B for either cache type): 8 KB of scratch, the epilogue
+// staging (2 KB per softmax warp) and, for e4m3, the two-entry P_lo ring (4 KB each),
+// which is never in use while a warp stages its epilogue (that waits for the split's
+// last PV; the next split's P is written by the same threads afterwards)
+constexpr uint32_t kOffScratch = 3 * 9 * 8192;
+static_assert(Geo<MLA_KV_BF16>::kStages * stage_bytes<MLA_KV_BF16>() == kOffScratch, "bf16 stages");
+static_assert(Geo<MLA_KV_E4M3>::kStages * stage_bytes<MLA_KV_E4M3>() == kOffScratch, "e4m3 stages");
 constexpr uint32_t kEpiWarpBytes = 16 * 128;
-constexpr uint32_t kOffBar = kOffEpi + 4 * kEpiWarpBytes;
-static_assert(kRows * kTok * 2 == kChunk, "P fills the rope chunk exactly");
+constexpr uint32_t kOffBar = kOffScratch + 8192;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory limit per block");
+static_assert(kRows * kTok * 2 == Geo<MLA_KV_BF16>::kChunk, "bf16 P fills the rope chunk exactly");
+static_assert(kRows * kTok == Geo<MLA_KV_E4M3>::kChunk, "e4m3 P_hi fills the rope chunk exactly");
 
 enum : int {
-    B_KV_FULL0 = 0, B_KV_EMPTY0 = B_KV_FULL0 + kStages, B_Q_FULL = B_KV_EMPTY0 + kStages, B_S_FULL0,
-    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_DRAIN = B_PV_DONE0 + 2, B_RAW0,
-    B_CONV = B_RAW0 + kStages, B_COUNT
+    B_KV_FULL0 = 0, B_KV_EMPTY0 = B_KV_FULL0 + kMaxStages, B_Q_FULL = B_KV_EMPTY0 + kMaxStages, B_S_FULL0,
+    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_DRAIN = B_PV_DONE0 + 2, B_COUNT
 };
 constexpr uint32_t kOffTmemHolder = kOffBar + 8 * B_COUNT;
 constexpr uint32_t kOffAbort = kOffTmemHolder + 4;
@@ -75,17 +111,23 @@ static_assert(kOffAbort + 4 <= kOffBar + 256, "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneHi = 16u << 16;  // second half-subpartition set (q and scores)
-constexpr uint32_t kColQ = 0;            // q: 288 columns (bf16 pairs)
+constexpr uint32_t kColQ = 0;            // q: 288 columns (bf16 pairs, or e4m3 q_hi | q_lo quads)
+constexpr uint32_t kColQlo = 144;        // e4m3 q_lo
 constexpr uint32_t kColS = 288;          // scores: 2 x 64 columns
-constexpr float kRescaleThreshold = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRows, kTok, 0, 0);
-constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kRows, 256, 0, 1);
+template <int KV>
+constexpr uint32_t idesc_s() {
+    return KV == MLA_KV_E4M3 ? ptx::idesc_e4m3_f32(kRows, kTok, 0, 0) : ptx::idesc_bf16_f32(kRows, kTok, 0, 0);
+}
+template <int KV>
+constexpr uint32_t idesc_pv() {
+    return KV == MLA_KV_E4M3 ? ptx::idesc_e4m3_f32(kRows, 256, 0, 1) : ptx::idesc_bf16_f32(kRows, 256, 0, 1);
+}
 
 struct __align__(64) Sm100Args {
     CUtensorMap tm_kv;  // cache viewed [P*64 rows, 576 cols]: bf16 box 64 x 64 with 128B swizzle, or
-                        // e4m3 box 64 x 64 bytes without swizzle
+                        // e4m3 box 64 x 64 bytes with 64B swizzle
     DecodeParams p;
 };
 
@@ -138,36 +180,44 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Twelve score K-steps starting at K0 (of 36): q from TMEM, the page from shared memory.
-// K0 is a template constant so that every descriptor offset is an immediate.
-template <int K0>
-__device__ __forceinline__ void issue_s_chunk(uint32_t d, uint32_t a0, uint64_t b0) {
-#pragma unroll
-    for (int k = 0; k < 12; ++k) {
-        constexpr int kChunkUnits = kChunk >> 4;
-        const int ks = K0 + k;
-        ptx::mma_ts(d, a0 + 8u * ks, b0 + (uint64_t)((ks >> 2) * kChunkUnits + (ks & 3) * 2), kIdescS,
-                    ks ? 1u : 0u);
-    }
+// Four floats -> (e4m3 word of x, e4m3 word of the residual x - e4m3(x)), bytes in order.
+__device__ __forceinline__ void split_e4m3x4(float x0, float x1, float x2, float x3, uint32_t& hi, uint32_t& lo) {
+    const uint16_t h01 = ptx::f32x2_to_e4m3x2(x0, x1), h23 = ptx::f32x2_to_e4m3x2(x2, x3);
+    const float2 f01 = e4m3x2_to_float2(h01), f23 = e4m3x2_to_float2(h23);
+    hi = (uint32_t)h01 | ((uint32_t)h23 << 16);
+    lo = (uint32_t)ptx::f32x2_to_e4m3x2(x0 - f01.x, x1 - f01.y) |
+         ((uint32_t)ptx::f32x2_to_e4m3x2(x2 - f23.x, x3 - f23.y) << 16);
 }
 
-// e4m3 -> bf16 for 32 consecutive bytes (exact: every e4m3 value is a bf16 value)
-__device__ __forceinline__ void widen_e4m3x32(const uint4 (&in)[2], uint32_t (&out)[16]) {
+// Twelve of the 36 score MMAs, starting at U0: q from TMEM, the page from shared memory.
+// U0 is a template constant so that every descriptor offset is an immediate.
+//   bf16: K-step u covers dims [16u, 16u + 16): chunk u / 4, 32-byte step u % 4 in the row.
+//   e4m3: term u / 18 (q_hi, q_lo), K-step v = u % 18 covers dims [32v, 32v + 32): chunk
+//         v / 2, 32-byte step v % 2 in the 64-byte row; q_lo starts 144 columns on.
+template <int KV, int U0>
+__device__ __forceinline__ void issue_s_chunk(uint32_t d, uint32_t a0, uint64_t b0) {
+    constexpr uint32_t kChunkUnits = Geo<KV>::kChunk >> 4;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        const uint32_t word = (w < 4) ? (&in[0].x)[w] : (&in[1].x)[w - 4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const float2 f = e4m3x2_to_float2((uint16_t)(word >> (16 * hh)));
-            __nv_bfloat162 v = __floats2bfloat162_rn(f.x, f.y);
-            out[2 * w + hh] = *reinterpret_cast<uint32_t*>(&v);
+    for (int k = 0; k < 12; ++k) {
+        const int u = U0 + k;
+        if constexpr (KV == MLA_KV_E4M3) {
+            const int v = u % 18;
+            ptx::mma_ts_f8(d, a0 + kColQlo * (uint32_t)(u / 18) + 8u * v,
+                           b0 + (uint64_t)((v >> 1) * kChunkUnits + (v & 1) * 2), idesc_s<KV>(), u ? 1u : 0u);
+        } else {
+            ptx::mma_ts(d, a0 + 8u * u, b0 + (uint64_t)((u >> 2) * kChunkUnits + (u & 3) * 2), idesc_s<KV>(),
+                        u ? 1u : 0u);
         }
     }
 }
 
 template <int KV>
-__global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(const __grid_constant__ Sm100Args args) {
+__global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_constant__ Sm100Args args) {
     constexpr bool kE4m3 = KV == MLA_KV_E4M3;
+    constexpr int kStages = Geo<KV>::kStages;
+    constexpr uint32_t kChunk = Geo<KV>::kChunk;
+    constexpr uint32_t kStageBytes = stage_bytes<KV>();
+    constexpr uint32_t kOffPInStage = 8 * kChunk;  // P (or P_hi) over the rope chunk
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
@@ -176,19 +226,8 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the combine may start its prologue now; it waits for this grid before reading
     ptx::griddep_launch_dependents();
-    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
-    // the plan (and every earlier write) must be complete before the header is read
-    ptx::griddep_wait();
 
-    if (h->magic != kPlanMagic || h->B != p.B || h->s_q != p.s_q || h->H != p.H ||
-        h->num_groups > p.groups_launched) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) set_status(h, kStatusPlanMismatch, 0);
-        return;
-    }
-    const int nqb = h->nqb;
-    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
-    if (g >= h->num_groups) return;
-
+    // prologue that reads no global memory, ahead of the wait for the grid before this one
     Ctx c;
     c.bar0 = sbase + kOffBar;
     c.abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
@@ -196,12 +235,9 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
     if (threadIdx.x == 0) {
         *c.abort = 0;
         for (int s = 0; s < kStages; ++s) {
-            // bf16: the TMA completes the stage; e4m3: the 128 converter threads do
-            ptx::mbar_init(c.bar(B_KV_FULL0 + s), kE4m3 ? 128 : 1);
+            ptx::mbar_init(c.bar(B_KV_FULL0 + s), 1);
             ptx::mbar_init(c.bar(B_KV_EMPTY0 + s), 1);
-            ptx::mbar_init(c.bar(B_RAW0 + s), 1);
         }
-        ptx::mbar_init(c.bar(B_CONV), 128);
         ptx::mbar_init(c.bar(B_Q_FULL), 128);
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(c.bar(B_S_FULL0 + s), 1);
@@ -211,6 +247,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
         ptx::mbar_init(c.bar(B_DRAIN), 1);
         ptx::fence_mbar_init_cluster();
     }
+    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
     if (warp == 1) {
         ptx::tmem_alloc(sbase + kOffTmemHolder, kTmemCols);
         ptx::tmem_relinquish();
@@ -219,6 +256,21 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemHolder);
+
+    // the plan (and every earlier write) must be complete before the header is read
+    ptx::griddep_wait();
+    const bool plan_ok = h->magic == kPlanMagic && h->B == p.B && h->s_q == p.s_q && h->H == p.H &&
+                         h->num_groups <= p.groups_launched;
+    const int nqb = plan_ok ? h->nqb : 1;
+    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
+    if (!plan_ok || g >= h->num_groups) {
+        if (!plan_ok && blockIdx.x == 0 && threadIdx.x == 0) set_status(h, kStatusPlanMismatch, 0);
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+        if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
 
     const int32_t* group_begin = ws_ptr<int32_t>(p.ws, h->off_group_begin);
     const Segment* segs = ws_ptr<Segment>(p.ws, h->off_segs);
@@ -254,19 +306,10 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                         // the softmax warps see the same id and poison the request's rows
                         const int ky = (page >= 0 && page < p.num_pages) ? page * kPage : -kPage;
                         const uint32_t dst = sbase + kOffKv + st * kStageBytes;
-                        if (kE4m3) {
-                            ptx::mbar_arrive_expect_tx(c.bar(B_RAW0 + st), kRawStageBytes);
+                        ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
 #pragma unroll
-                            for (int jb = 0; jb < 9; ++jb)
-                                ptx::tma_load_2d(dst + jb * kChunk + kRawChunk, &args.tm_kv, c.bar(B_RAW0 + st),
-                                                 64 * jb, ky);
-                        } else {
-                            ptx::mbar_arrive_expect_tx(c.bar(B_KV_FULL0 + st), kStageBytes);
-#pragma unroll
-                            for (int jb = 0; jb < 9; ++jb)
-                                ptx::tma_load_2d(dst + jb * kChunk, &args.tm_kv, c.bar(B_KV_FULL0 + st), 64 * jb,
-                                                 ky);
-                        }
+                        for (int jb = 0; jb < 9; ++jb)
+                            ptx::tma_load_2d(dst + jb * kChunk, &args.tm_kv, c.bar(B_KV_FULL0 + st), 64 * jb, ky);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -275,7 +318,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
         }
         if (lane == 0 && *c.abort) {
             for (int k = (it > kStages ? it - kStages : 0); k < it; ++k)
-                drain_wait(c.bar((kE4m3 ? B_RAW0 : B_KV_FULL0) + k % kStages), (k / kStages) & 1);
+                drain_wait(c.bar(B_KV_FULL0 + k % kStages), (k / kStages) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -307,13 +350,13 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                             ptx::tc_fence_after();
                             // descriptors are built once and advanced by constant 16-byte offsets:
                             // the fully unrolled issue loop is a handful of integer adds per MMA
-                            const uint64_t b0 = ptx::smem_desc(sbase + kOffKv + st * kStageBytes, 16, 1024,
-                                                               ptx::kSwizzle128);
+                            const uint64_t b0 = ptx::smem_desc(sbase + kOffKv + st * kStageBytes, 16, Geo<KV>::kSbo,
+                                                               Geo<KV>::kSwizzle);
                             const uint32_t d = tmem + kLaneHi + kColS + 64u * (its & 1);
                             const uint32_t a0 = tmem + kLaneHi + kColQ;
-                            issue_s_chunk<0>(d, a0, b0);
-                            issue_s_chunk<12>(d, a0, b0);
-                            issue_s_chunk<24>(d, a0, b0);
+                            issue_s_chunk<KV, 0>(d, a0, b0);
+                            issue_s_chunk<KV, 12>(d, a0, b0);
+                            issue_s_chunk<KV, 24>(d, a0, b0);
                             ptx::mma_commit(c.bar(B_S_FULL0 + (its & 1)));
                             ++ns;
                             progressed = true;
@@ -324,18 +367,33 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                         if (ptx::mbar_test_wait(c.bar(B_P_READY0 + (itp & 1)), (itp >> 1) & 1)) {
                             ptx::tc_fence_after();
                             const bool first = npv == 0;
-                            // A = P (K-major); B = V, MN-major: 64-column blocks 8 KB apart (leading
-                            // offset), 8-token groups 1 KB apart (stride offset)
+                            // A = P (K-major); B = V, MN-major: 64-column chunks one chunk apart
+                            // (leading offset), 8-token groups one swizzle atom apart (stride offset)
                             const uint32_t stage = sbase + kOffKv + (itp % kStages) * kStageBytes;
-                            const uint64_t a0 = ptx::smem_desc(stage + kOffPInStage, 16, 1024, ptx::kSwizzle128);
-                            const uint64_t v0 = ptx::smem_desc(stage, kChunk, 1024, ptx::kSwizzle128);
+                            const uint64_t v0 = ptx::smem_desc(stage, kChunk, Geo<KV>::kSbo, Geo<KV>::kSwizzle);
+                            if constexpr (kE4m3) {
+                                const uint64_t ph = ptx::smem_desc(stage + kOffPInStage, 16, 512, ptx::kSwizzle64);
+                                const uint64_t pl =
+                                    ptx::smem_desc(sbase + kOffScratch + 4096u * (itp & 1), 16, 512, ptx::kSwizzle64);
 #pragma unroll
-                            for (int half = 0; half < 2; ++half) {
+                                for (int term = 0; term < 2; ++term)
 #pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
-                                    ptx::mma_ss(tmem + 256u * half, a0 + (uint64_t)(ks * 2),
-                                                v0 + (uint64_t)(half * 4 * (kChunk >> 4) + ks * (2048 >> 4)), kIdescPV,
-                                                (first && ks == 0) ? 0u : 1u);
+                                    for (int half = 0; half < 2; ++half)
+#pragma unroll
+                                        for (int ks = 0; ks < 2; ++ks)  // 32 tokens: 32 bytes of P, 2 KB of V
+                                            ptx::mma_ss_f8(tmem + 256u * half, (term ? pl : ph) + (uint64_t)(ks * 2),
+                                                           v0 + (uint64_t)(half * 4 * (kChunk >> 4) + ks * (2048 >> 4)),
+                                                           idesc_pv<KV>(), (first && term == 0 && ks == 0) ? 0u : 1u);
+                            } else {
+                                const uint64_t a0 = ptx::smem_desc(stage + kOffPInStage, 16, 1024, ptx::kSwizzle128);
+#pragma unroll
+                                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                                    for (int ks = 0; ks < 4; ++ks)  // 16 tokens: 32 bytes of P, 2 KB of V
+                                        ptx::mma_ss(tmem + 256u * half, a0 + (uint64_t)(ks * 2),
+                                                    v0 + (uint64_t)(half * 4 * (kChunk >> 4) + ks * (2048 >> 4)),
+                                                    idesc_pv<KV>(), (first && ks == 0) ? 0u : 1u);
+                                }
                             }
                             ptx::mma_commit(c.bar(B_PV_DONE0 + (itp & 1)));
                             ptx::mma_commit(c.bar(B_KV_EMPTY0 + (itp % kStages)));
@@ -365,50 +423,6 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             }
             ptx::mma_commit(c.bar(B_DRAIN));
             drain_wait(c.bar(B_DRAIN), 0);
-        }
-    } else if (kE4m3 && warp >= 6) {
-        // ------------------------------------------------------------ e4m3 -> bf16 (warps 6-9)
-        // Every thread takes one half-row (32 bytes) of each of the nine chunks: all reads
-        // first, a bounded barrier among the converters, then the writes, because each bf16
-        // chunk overwrites its own e4m3 bytes in the upper half of its slot.
-        const int ct = threadIdx.x - 192;  // 0..127
-        const int r = ct >> 1, hf = ct & 1;
-        int it = 0;
-        bool alive = true;
-        for (int si = seg_lo; si < seg_hi && alive; ++si) {
-            const Segment S = segs[si];
-            const int T = p.seq_lens[S.b];
-            if (!request_ok(p, T)) continue;
-            for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
-                const int st = it % kStages;
-                alive = wait_bar(c, c.bar(B_RAW0 + st), (it / kStages) & 1);
-                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
-                uint8_t* stage = smem + kOffKv + st * kStageBytes;
-                uint4 raw[9][2];
-#pragma unroll
-                for (int j = 0; j < 9; ++j) {
-                    const uint4* src = reinterpret_cast<const uint4*>(stage + j * kChunk + kRawChunk + r * 64 + hf * 32);
-                    raw[j][0] = src[0];
-                    raw[j][1] = src[1];
-                }
-                ptx::mbar_arrive(c.bar(B_CONV));
-                alive = wait_bar(c, c.bar(B_CONV), it & 1);
-                if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
-#pragma unroll
-                for (int j = 0; j < 9; ++j) {
-                    uint32_t o[16];
-                    widen_e4m3x32(raw[j], o);
-                    uint8_t* rowp = stage + j * kChunk + r * 128;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const int piece = 4 * hf + w;  // 16-byte piece of the 128-byte row, swizzled
-                        *reinterpret_cast<uint4*>(rowp + ((piece ^ (r & 7)) << 4)) =
-                            make_uint4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
-                    }
-                }
-                ptx::fence_proxy_async_smem();
-                ptx::mbar_arrive(c.bar(B_KV_FULL0 + st));
-            }
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
@@ -453,24 +467,72 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 continue;
             }
             if (*c.abort) break;
-            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row.
-            // The loads of a batch are all issued before the first is used: at a split's start
-            // the memory system is full of the first pages' loads, and every dependent round
-            // trip here delays the first score MMA.  One batch of 36 loads per thread; three
-            // for an e4m3 cache, whose kernel has fewer registers per thread.
+            // q rows of this block into TMEM.  Thread (row, half) holds dims [64 k + 32 half,
+            // +32) for k = 0..8, loaded in one batch of 36 16-byte loads (all issued before the
+            // first is used: at a split's start the memory system is full of the first pages'
+            // loads, and every dependent round trip here delays the first score MMA).
+            // For an e4m3 cache the row is cut into two e4m3 terms at one per-row scale
+            // s_r = max|q_r| / 448, which multiplies the row's scores.
+            float row_scale = 1.f;
             {
-                constexpr int kQBatch = kE4m3 ? 3 : 9;  // column blocks per batch
                 const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + m_glob) * kDqk);
+                uint4 x[9][4];
+#pragma unroll
+                for (int k = 0; k < 9; ++k)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        x[k][w] = row_valid ? src[(64 * k + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
+                if constexpr (kE4m3) {
+                    // first pass: the row's max |q| (both halves); second pass: each 32-dim
+                    // block loaded again (an L1 hit) and split into its two e4m3 terms, so that
+                    // the loaded row and its terms are never live together
+                    float amax = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 9; ++k)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t v4[4] = {x[k][w].x, x[k][w].y, x[k][w].z, x[k][w].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(v4[e] << 16)),
+                                                         fabsf(__uint_as_float(v4[e] & 0xffff0000u))));
+                        }
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+                    // the largest power of two 2^k with max|q| 2^k <= 448: q 2^k is still a
+                    // bf16 value (8 significant bits), which the two e4m3 terms (4 + 4 bits)
+                    // hold exactly unless it is small enough for e4m3's subnormal range
+                    float inv = 0.f;
+                    row_scale = 0.f;
+                    if (amax > 0.f) {
+                        int e;
+                        const float f = frexpf(amax, &e);  // amax = f 2^e, f in [0.5, 1)
+                        const int k = min(127, max(-126, (f <= 0.875f ? 9 : 8) - e));
+                        inv = ldexpf(1.f, k);
+                        row_scale = ldexpf(1.f, -k);
+                    }
 #pragma unroll 1
-                for (int kb = 0; kb < 9; kb += kQBatch) {
-                    uint4 x[kQBatch][4];
+                    for (int k = 0; k < 9; ++k) {
+                        uint4 y[4];
 #pragma unroll
-                    for (int k = 0; k < kQBatch; ++k)
+                        for (int w = 0; w < 4; ++w)
+                            y[w] = row_valid ? src[(64 * k + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
+                        uint32_t hi[8], lo[8];
 #pragma unroll
-                        for (int w = 0; w < 4; ++w)  // dims [64 (kb + k) + 32 half, +32)
-                            x[k][w] = row_valid ? src[(64 * (kb + k) + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t v4[4] = {y[w].x, y[w].y, y[w].z, y[w].w};
 #pragma unroll
-                    for (int k = 0; k < kQBatch; ++k) {
+                            for (int e = 0; e < 4; e += 2)
+                                split_e4m3x4(__uint_as_float(v4[e] << 16) * inv, __uint_as_float(v4[e] & 0xffff0000u) * inv,
+                                             __uint_as_float(v4[e + 1] << 16) * inv,
+                                             __uint_as_float(v4[e + 1] & 0xffff0000u) * inv, hi[2 * w + e / 2],
+                                             lo[2 * w + e / 2]);
+                        }
+                        ptx::tmem_st16x8<8>(t_hi + kColQ + 16u * k, hi);
+                        ptx::tmem_st16x8<8>(t_hi + kColQlo + 16u * k, lo);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 9; ++k) {
                         uint32_t v[16];
 #pragma unroll
                         for (int w = 0; w < 4; ++w) {
@@ -479,7 +541,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                             v[4 * w + 2] = x[k][w].z;
                             v[4 * w + 3] = x[k][w].w;
                         }
-                        ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * (kb + k), v);
+                        ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * k, v);
                     }
                 }
                 ptx::tmem_wait_st();
@@ -490,6 +552,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             const int full_end = p.causal ? T - p.s_q + 1 : T;  // tokens < full_end are visible to every row
             const int ntiles_req = (T + kPage - 1) / kPage;
             const int n = S.tile_end - S.tile_begin;
+            const float sc = p.score_scale_log2 * row_scale;
             float m_run = -INFINITY, l = 0.f;
             bool badpage = false;
             for (int jj = 0; jj < n; ++jj, ++it) {
@@ -503,7 +566,6 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 ptx::tmem_ld16x32<32>(t_hi + kColS + 64u * (it & 1), sr);
                 ptx::tmem_wait_ld();
                 float s[32];
-                const float sc = p.score_scale_log2;
                 const int tok0 = tile * kPage + 32 * half;
                 if (tile * kPage + kPage <= full_end) {
 #pragma unroll
@@ -522,7 +584,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
                 float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                const bool raise = mt > m_run + kRescaleThreshold;
+                const bool raise = mt > m_run + Geo<KV>::kRescale;
                 float alpha = 1.f;
                 if (raise) {
                     alpha = fast_exp2(m_run - mt);
@@ -547,37 +609,56 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                     }
                     ptx::tmem_wait_st();
                 }
-                uint32_t pk[16];
-                float rs[4] = {0.f, 0.f, 0.f, 0.f};
                 const bool live = m_run != -INFINITY;
+                const float mo = m_run - Geo<KV>::kPOffset;  // P = 2^(x - m + offset)
+                float pv[32];
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float p0 = live ? fast_exp2(s[2 * k] - m_run) : 0.f;
-                    const float p1 = live ? fast_exp2(s[2 * k + 1] - m_run) : 0.f;
-                    rs[k & 3] += p0 + p1;
-                    pk[k] = pack_bf16(p0, p1);
+                for (int k = 0; k < 32; ++k) {
+                    pv[k] = live ? fast_exp2(s[k] - mo) : 0.f;
+                    rs[(k >> 1) & 3] += pv[k];
                 }
                 l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+                uint8_t* stage_p = smem + kOffKv + (it % kStages) * kStageBytes;
                 if (tile == ntiles_req - 1 && (T % kPage) != 0) {
                     // rows past the request's end hold stale data (maybe NaN): zero their
                     // latent columns before the PV product reads them with P = 0
                     alive = wait_bar(c, c.bar(B_KV_FULL0 + it % kStages), (it / kStages) & 1);
                     if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
                     const int r0 = T % kPage;
-                    uint8_t* vb = smem + kOffKv + (it % kStages) * kStageBytes;
-                    const int pieces = (kPage - r0) * 8 * 8;  // rows x latent chunks x 16-byte pieces
+                    constexpr int kPieces = (int)(kChunk / kTok / 16);  // 16-byte pieces per chunk row
+                    const int pieces = (kPage - r0) * 8 * kPieces;      // rows x latent chunks x pieces
                     for (int q = tid; q < pieces; q += 128) {
-                        const int r = r0 + q / 64, j = (q / 8) % 8, w = q % 8;
-                        *reinterpret_cast<uint4*>(vb + j * kChunk + r * 128 + w * 16) = make_uint4(0, 0, 0, 0);
+                        const int r = r0 + q / (8 * kPieces), j = (q / kPieces) % 8, w = q % kPieces;
+                        *reinterpret_cast<uint4*>(stage_p + j * kChunk + r * (kChunk / kTok) + w * 16) =
+                            make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();
                 }
-                {
+                if constexpr (kE4m3) {
+                    // P_hi over the rope chunk, P_lo into the ring: row `row`, tokens [32 half,
+                    // +32): two 16-byte pieces of the 64-byte K-major row, 64-byte swizzle
+                    // (piece c of row r at (c ^ ((r >> 1) & 3)) * 16)
+                    uint32_t hi[8], lo[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        split_e4m3x4(pv[4 * k], pv[4 * k + 1], pv[4 * k + 2], pv[4 * k + 3], hi[k], lo[k]);
+                    uint8_t* ph = stage_p + kOffPInStage + row * 64;
+                    uint8_t* pl = smem + kOffScratch + 4096 * (it & 1) + row * 64;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const int off = ((2 * half + w) ^ ((row >> 1) & 3)) << 4;
+                        *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[4 * w], hi[4 * w + 1], hi[4 * w + 2], hi[4 * w + 3]);
+                        *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[4 * w], lo[4 * w + 1], lo[4 * w + 2], lo[4 * w + 3]);
+                    }
+                } else {
                     // P row `row`, tokens [32 half, 32 half + 32): four 16-byte chunks of the
                     // 128-byte K-major row, 128-byte swizzle, over the page's rope chunk (the
                     // score MMAs that read it have completed: S_FULL was waited above)
-                    uint8_t* pbuf = smem + kOffKv + (it % kStages) * kStageBytes + kOffPInStage;
-                    uint8_t* prow_s = pbuf + (row >> 3) * 1024 + (row & 7) * 128;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) pk[k] = pack_bf16(pv[2 * k], pv[2 * k + 1]);
+                    uint8_t* prow_s = stage_p + kOffPInStage + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         const int chunk = 4 * half + w;
@@ -603,7 +684,7 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
             // warp covers two whole 256-byte runs.  A request held whole goes to the bf16
             // output, row-major, through a 2 KB staging tile per warp (16 rows x 128 bytes,
             // 16-byte pieces XOR-swizzled by row) so that every store writes whole row segments.
-            uint8_t* stg = smem + kOffEpi + (warp - 2) * kEpiWarpBytes;
+            uint8_t* stg = smem + kOffScratch + (warp - 2) * kEpiWarpBytes;
             const int rows_ok = min(16, p.M - (qb * kRows + quad * 16));  // valid rows of this warp
             const int64_t out_row0 = (int64_t)S.b * p.M + qb * kRows + quad * 16;
             float4* pq = reinterpret_cast<float4*>(po + ((int64_t)si * nqb + qb) * kRows * kDv) + quad * 2048 +
@@ -654,7 +735,8 @@ __global__ void __launch_bounds__(threads_for<KV>(), 1) decode_sm100_kernel(cons
                 store_chunk(q + 1, ob);
             }
             if (row_valid && half == 0) {
-                const float lse2 = badpage ? nanv : (l > 0.f ? m_run + __log2f(l) : -INFINITY);
+                const float lse2 =
+                    badpage ? nanv : (l > 0.f ? m_run - Geo<KV>::kPOffset + __log2f(l) : -INFINITY);
                 if (!S.split)
                     p.lse[orow] = lse2 * kLn2;
                 else
@@ -710,7 +792,7 @@ int sm100_cta_slots() {
                              (int)kSmemBytes) != cudaSuccess)
         return -1;
     int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_sm100_kernel<MLA_KV_E4M3>, kThreadsE4m3,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_sm100_kernel<MLA_KV_E4M3>, kThreads,
                                                       kSmemBytes) !=
             cudaSuccess ||
         per_sm <= 0)
@@ -738,7 +820,7 @@ bool cached_kv_map(int dev, const DecodeParams& p, CUtensorMap* out) {
         const uint64_t kvrows = (uint64_t)p.num_pages * kPage;
         const bool ok = KV == MLA_KV_E4M3
                             ? make_map_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.kv, kDqk, kvrows, kDqk, 64, kTok,
-                                          CU_TENSOR_MAP_SWIZZLE_NONE)
+                                          CU_TENSOR_MAP_SWIZZLE_64B)
                             : make_map_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.kv, kDqk, kvrows, kDqk * 2, 64,
                                           kTok, CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) {
@@ -780,7 +862,7 @@ mla_status launch_typed(const DecodeParams& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(ctas);
-    cfg.blockDim = dim3(threads_for<KV>());
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
