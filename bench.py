@@ -51,7 +51,9 @@ DEFAULT_WORKLOAD = "long_m256"  # the largest single-GPU configuration: B=16, s_
 METRIC = "MLA decode \u00b5s/call and KV-read GB/s (% of B200 HBM/tensor roofline)"  # value in GB/s; us_per_call beside it
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # B200 datasheet (dense bf16), for context
-KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_sm100.cu"]
+KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_sm100.cu",
+                  "mla_attention_decode_paged_b200/csrc/mla_decode_sm100_e4m3.cu",
+                  "mla_attention_decode_paged_b200/csrc/mla_scan_common.cuh"]
 
 
 def log(*a):
