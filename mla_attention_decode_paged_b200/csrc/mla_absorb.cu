@@ -6,137 +6,234 @@
 //     q[r, h, 0:512]   = W_UK[h] q_nope[r, h]      (so that q . c = q_nope . k_nope)
 //     q[r, h, 512:576] = q_rope[r, h]              (the decoupled rope part, copied)
 //     y[r, h, :]       = out[r, h, :] W_UV[h]      (128 wide)
-// Both are a batched GEMM over heads, Y_h = X_h B_h with B_h = W_UK[h]^T (K = 128,
-// N = 512) or W_UV[h] (K = 512, N = 128), and R = B * s_q rows per head.  At decode
-// sizes (R = 16..256) the weights dominate the bytes (128 KB per head and matrix); the
-// contraction runs on the CUDA cores in fp32 (16 rows per CTA are too few for a 64- or
-// 128-row tensor-core tile) and the result is rounded to bf16 (nearest, ties to even).
-#include <math.h>
+//
+// Both are batched GEMMs over heads with R = B * s_q rows per head, run on the tcgen05
+// tensor cores in the transposed form D_h = A_h X_h^T, so that the MMA's 128-row M side
+// is the weight's dimension (a full-rate tile at any R) and the rows r are its N side:
+//     project: D[c, r] = sum_d W_UV[h][d][c] out[r, h, d]   M = 128 (c), K = 512 (d)
+//              A = W_UV[h] read MN-major (c contiguous in memory)
+//     absorb:  D[d, r] = sum_k W_UK[h][d][k] q_nope[r, h, k]   M = 512 (d, four tiles), K = 128
+//              A = W_UK[h] read K-major (k contiguous)
+// X_h^T is K-major in both (a row's K values are contiguous).  One CTA per (head, M tile,
+// N tile of up to 256 rows): TMA brings 64-wide K chunks of A (128 x 64) and X (N x 64)
+// into 128B-swizzled shared memory, in up to four stages; one thread issues the MMAs
+// (M=128, N, K=16) into a TMEM accumulator of N fp32 columns; then the four warps read it
+// back (warp w: lanes 32w..32w+31, i.e. 32 values of the M side) and write bf16 (nearest,
+// ties to even).  The X boxes are three-dimensional, [K chunk, 1 head, N rows], so one
+// head's rows land as a dense N x 128-byte tile.  Rows past R read as zeros (the box runs
+// off the tensor) and are not written.
+#include <cudaTypedefs.h>
+#include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "mla_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
 
-constexpr int kBN = 32;              // output columns per CTA
-constexpr int kRB = 16;              // query rows per CTA
-constexpr int kAbsorbThreads = 256;  // 8 warps, each a slice of the contraction
-constexpr int kKWarps = kAbsorbThreads / 32;
+constexpr int kGemmThreads = 128;
+constexpr int kKChunk = 64;                       // K per stage: one 128-byte swizzle row of bf16
+constexpr int kMaxStages = 4;
+constexpr uint32_t kATile = 128 * kKChunk * 2;    // 16 KB
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Y[r, h, n] (row stride y_rs, head stride y_hs) = sum_k X[r, h, k] * B_h[k, n], with
-// X[r, h, k] at x + r * x_rs + h * K + k and B_h[k, n] at w + h * K * N + (B_T ? n * K + k
-// : k * N + n).  A CTA takes 32 output columns of one head and every gridDim.z-th block of
-// 16 rows: the weight tile (K x 32, read once with 16-byte loads, all in flight together)
-// and each block's rows go to shared memory;
-// each warp contracts one eighth of K for the whole 16 x 32 tile (a lane holds a 4 x 4
-// block: 16 independent accumulators), and the eight partial tiles are added in shared
-// memory.
-template <bool B_T, int K, int N>
-__global__ void __launch_bounds__(kAbsorbThreads) head_gemm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_rs,
-                                                                  const __nv_bfloat16* __restrict__ w,
-                                                                  __nv_bfloat16* __restrict__ y, int64_t y_rs,
-                                                                  int64_t y_hs, int R,
-                                                                  const __nv_bfloat16* __restrict__ rope) {
-    extern __shared__ __align__(16) uint8_t absorb_smem[];
-    __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(absorb_smem);                 // [K][kBN]
-    float* xs = reinterpret_cast<float*>(absorb_smem + K * kBN * 2);                    // [K][kRB]
-    float* red = xs + K * kRB;                                                          // [kKWarps][kRB][kBN]
-    const int n0 = blockIdx.x * kBN, h = blockIdx.y;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const __nv_bfloat16* wh = w + (int64_t)h * K * N;
-    if (B_T) {
-        // rows n0..n0+31 of W (K contiguous values each), transposed into wt[k][n]
-        for (int e = tid; e < kBN * (K / 8); e += kAbsorbThreads) {
-            const int nn = e / (K / 8), k8 = e % (K / 8);
-            const uint4 v = *reinterpret_cast<const uint4*>(wh + (int64_t)(n0 + nn) * K + 8 * k8);
-            const __nv_bfloat16* pv = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) wt[(8 * k8 + j) * kBN + nn] = pv[j];
-        }
-    } else {
-        // columns n0..n0+31 of each of the K rows (64 contiguous bytes per row)
-        for (int e = tid; e < K * (kBN / 8); e += kAbsorbThreads) {
-            const int kk = e / (kBN / 8), c8 = e % (kBN / 8);
-            *reinterpret_cast<uint4*>(wt + kk * kBN + 8 * c8) =
-                *reinterpret_cast<const uint4*>(wh + (int64_t)kk * N + n0 + 8 * c8);
-        }
-    }
-    // row blocks blockIdx.z, blockIdx.z + gridDim.z, ...: the weight tile is loaded once
-    for (int r0 = blockIdx.z * kRB; r0 < R; r0 += gridDim.z * kRB) {
-        __syncthreads();  // the previous block's rows and partial tiles are consumed
-        // the block's 16 rows, transposed to xs[k][row] in fp32
-        for (int e = tid; e < kRB * (K / 8); e += kAbsorbThreads) {
-            const int rr = e / (K / 8), k8 = e % (K / 8);
-            const int r = r0 + rr;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (r < R) v = *reinterpret_cast<const uint4*>(x + (int64_t)r * x_rs + (int64_t)h * K + 8 * k8);
-            const __nv_bfloat16* pv = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) xs[(8 * k8 + j) * kRB + rr] = __bfloat162float(pv[j]);
-        }
-        if (rope && blockIdx.x == 0) {
-            // the query's rope part: y[r, h, 512:576] = rope[r, h, :] for this CTA's rows
-            for (int e = tid; e < kRB * 8; e += kAbsorbThreads) {
-                const int rr = e >> 3, p8 = e & 7, r = r0 + rr;
-                if (r < R)
-                    *reinterpret_cast<uint4*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + kDv + 8 * p8) =
-                        *reinterpret_cast<const uint4*>(rope + ((int64_t)r * gridDim.y + h) * 64 + 8 * p8);
+struct __align__(64) GemmArgs {
+    CUtensorMap tm_a;   // the weights: project {128 c, 512 d, H} box {64, 64, 1}; absorb {128 k, 512 d, H} box {64, 128, 1}
+    CUtensorMap tm_x;   // the rows: {K, H, R} box {64, 1, N}
+    __nv_bfloat16* y;   // output rows: y[r * y_rs + h * y_hs + m]
+    int64_t y_rs, y_hs;
+    const __nv_bfloat16* rope;  // absorb only: q_rope [R, H, 64], copied to y[..., 512:576]
+    int R, H, N;        // rows, heads, N tile (a multiple of 16, <= 256)
+    int32_t* status;    // where a bounded wait that gave up is recorded (may be null)
+};
+
+// Bounded mbarrier wait (2 s); false if it gave up.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int32_t* status) {
+    uint64_t t0 = 0;
+    for (uint32_t n = 1;; ++n) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((n & 255) == 0) {
+            const uint64_t now = ptx::globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+                if (status) atomicCAS(status, 0, (int32_t)kStatusTimeout);
+                return false;
             }
-        }
-        __syncthreads();
-        const int rg = lane >> 3, cg = lane & 7;  // rows 4 rg .. 4 rg + 3, columns 4 cg .. 4 cg + 3
-        float acc[4][4] = {};
-        constexpr int kSlice = K / kKWarps;
-#pragma unroll 4
-        for (int kk = warp * kSlice; kk < (warp + 1) * kSlice; ++kk) {
-            const float4 xv = *reinterpret_cast<const float4*>(xs + kk * kRB + 4 * rg);
-            const uint2 wb = *reinterpret_cast<const uint2*>(wt + kk * kBN + 4 * cg);
-            const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.x));
-            const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb.y));
-            const float xr[4] = {xv.x, xv.y, xv.z, xv.w}, wc[4] = {w01.x, w01.y, w23.x, w23.y};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xr[i], wc[j], acc[i][j]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(red + (warp * kRB + 4 * rg + i) * kBN + 4 * cg) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        __syncthreads();
-        // the eight partial tiles, added in warp order (a fixed order: deterministic)
-        for (int o = tid; o < kRB * kBN / 2; o += kAbsorbThreads) {
-            const int rr = o / (kBN / 2), c = 2 * (o % (kBN / 2));
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int q = 0; q < kKWarps; ++q) {
-                s0 += red[(q * kRB + rr) * kBN + c];
-                s1 += red[(q * kRB + rr) * kBN + c + 1];
-            }
-            const int r = r0 + rr;
-            if (r < R)
-                *reinterpret_cast<__nv_bfloat162*>(y + (int64_t)r * y_rs + (int64_t)h * y_hs + n0 + c) =
-                    __floats2bfloat162_rn(s0, s1);
         }
     }
 }
 
-template <bool B_T, int K, int N>
-cudaError_t launch_head_gemm(const __nv_bfloat16* x, int64_t x_rs, const __nv_bfloat16* w, __nv_bfloat16* y,
-                             int64_t y_rs, int64_t y_hs, int R, int H, const __nv_bfloat16* rope, cudaStream_t st) {
-    constexpr int kSmem = K * kBN * 2 + K * kRB * 4 + kKWarps * kRB * kBN * 4;
-    if (kSmem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(head_gemm_kernel<B_T, K, N>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        if (e != cudaSuccess) return e;
+// kK: the contraction length (512 project, 128 absorb); kAMn: A read MN-major (project).
+template <int kK, bool kAMn>
+__global__ void __launch_bounds__(kGemmThreads, 1) head_gemm_sm100_kernel(const __grid_constant__ GemmArgs g) {
+    constexpr int kChunks = kK / kKChunk;
+    constexpr int kStages = kChunks < kMaxStages ? kChunks : kMaxStages;
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int h = blockIdx.x, mt = blockIdx.y, n0 = blockIdx.z * g.N;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t x_tile = (uint32_t)g.N * 128;        // N rows x 64 bf16
+    const uint32_t stage_bytes = kATile + x_tile;
+    const uint32_t off_bar = kStages * stage_bytes;      // full[kStages], empty[kStages], done
+    auto bar = [&](int i) { return sbase + off_bar + 8u * (uint32_t)i; };
+    const uint32_t holder = off_bar + 8u * (2 * kStages + 1);
+    uint32_t ncols = 32;
+    while ((int)ncols < g.N) ncols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar(s), 1);
+            ptx::mbar_init(bar(kStages + s), 1);
+        }
+        ptx::mbar_init(bar(2 * kStages), 1);
+        ptx::fence_mbar_init_cluster();
+        ptx::prefetch_tmap(&g.tm_a);
+        ptx::prefetch_tmap(&g.tm_x);
     }
-    // at most four CTAs share a (head, column tile): each reads the weight tile once
-    const int zblocks = std::min((R + kRB - 1) / kRB, 4);
-    head_gemm_kernel<B_T, K, N><<<dim3(N / kBN, H, zblocks), kAbsorbThreads, kSmem, st>>>(
-        x, x_rs, w, y, y_rs, y_hs, R, rope);
-    return cudaGetLastError();
+    if (warp == 1) {
+        ptx::tmem_alloc(sbase + holder, ncols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + holder);
+    bool ok = true;
+
+    if (warp == 0 && lane == 0) {
+        // producer: chunk c into stage c % kStages, once the MMAs of chunk c - kStages are done
+        for (int c = 0; c < kChunks && ok; ++c) {
+            const int s = c % kStages;
+            if (c >= kStages && !wait_bounded(bar(kStages + s), ((c / kStages) - 1) & 1, g.status)) {
+                ok = false;
+                break;
+            }
+            const uint32_t a_dst = sbase + s * stage_bytes, x_dst = a_dst + kATile;
+            ptx::mbar_arrive_expect_tx(bar(s), stage_bytes);
+            if (kAMn) {
+                // W_UV[h] rows d in [64 c, +64), columns c in [0, 64) and [64, 128): two 8 KB
+                // MN-major atoms (64 columns x 64 rows of 128 bytes)
+                ptx::tma_load_3d(a_dst, &g.tm_a, bar(s), 0, kKChunk * c, h);
+                ptx::tma_load_3d(a_dst + kATile / 2, &g.tm_a, bar(s), 64, kKChunk * c, h);
+            } else {
+                // W_UK[h] rows d in [128 mt, +128), columns k in [64 c, +64): K-major 128 x 128 B
+                ptx::tma_load_3d(a_dst, &g.tm_a, bar(s), kKChunk * c, 128 * mt, h);
+            }
+            ptx::tma_load_3d(x_dst, &g.tm_x, bar(s), kKChunk * c, h, n0);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: four K=16 steps per chunk into one accumulator
+        const uint32_t idesc = ptx::idesc_bf16_f32(128, g.N, kAMn ? 1 : 0, 0);
+        for (int c = 0; c < kChunks && ok; ++c) {
+            const int s = c % kStages;
+            if (!wait_bounded(bar(s), (c / kStages) & 1, g.status)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t a_src = sbase + s * stage_bytes, x_src = a_src + kATile;
+            // MN-major A: 64-column atoms 8 KB apart (leading), 8 K-rows 1 KB apart (stride);
+            // K-major A and X: 8 rows 1 KB apart (stride)
+            const uint64_t a0 = kAMn ? ptx::smem_desc(a_src, kATile / 2, 1024, ptx::kSwizzle128)
+                                     : ptx::smem_desc(a_src, 16, 1024, ptx::kSwizzle128);
+            const uint64_t x0 = ptx::smem_desc(x_src, 16, 1024, ptx::kSwizzle128);
+#pragma unroll
+            for (int ks = 0; ks < kKChunk / 16; ++ks) {
+                // K step: 16 values = 32 bytes along a K-major row, or 16 rows = 2 KB of an
+                // MN-major atom
+                const uint64_t a = a0 + (uint64_t)(kAMn ? ks * (2048 >> 4) : ks * 2);
+                ptx::mma_ss(tmem, a, x0 + (uint64_t)(ks * 2), idesc, (c | ks) ? 1u : 0u);
+            }
+            ptx::mma_commit(bar(kStages + s));
+        }
+        ptx::mma_commit(bar(2 * kStages));
+    }
+    __syncwarp();
+    // epilogue: every warp waits for the last MMA, then reads its 32 lanes (M side)
+    const bool done = wait_bounded(bar(2 * kStages), 0, g.status);
+    ptx::tc_fence_after();
+    if (done) {
+        const int m = 128 * mt + 32 * warp + lane;  // the output column this thread writes
+        const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+        for (int c0 = 0; c0 < g.N; c0 += 16) {
+            uint32_t v[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                "%13, %14, %15}, [%16];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                : "r"(t_row + (uint32_t)c0)
+                : "memory");
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = n0 + c0 + j;
+                if (r < g.R) g.y[(int64_t)r * g.y_rs + (int64_t)h * g.y_hs + m] = __float2bfloat16_rn(__uint_as_float(v[j]));
+            }
+        }
+        if (g.rope && mt == 0) {
+            // the query's rope part: y[r, h, 512:576] = q_rope[r, h, :] for this CTA's rows
+            for (int e = threadIdx.x; e < g.N * 8; e += kGemmThreads) {
+                const int r = n0 + (e >> 3), p8 = e & 7;
+                if (r < g.R)
+                    *reinterpret_cast<uint4*>(g.y + (int64_t)r * g.y_rs + (int64_t)h * g.y_hs + kDv + 8 * p8) =
+                        *reinterpret_cast<const uint4*>(g.rope + ((int64_t)r * g.H + h) * 64 + 8 * p8);
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem, ncols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// A 3-D bf16 tensor map: dims {d0, d1, d2} (d0 contiguous), byte strides of d1 and d2,
+// box {b0, b1, b2}, 128-byte swizzle (b0 * 2 bytes = 128).
+bool map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+            uint32_t b0, uint32_t b1, uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1, s2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// N tile: R rounded up to 16, at most 256 (the TMEM columns of one accumulator).
+int n_tile(int R) { return std::min(256, (R + 15) / 16 * 16); }
+
+template <int kK, bool kAMn>
+mla_status launch_head_gemm(const GemmArgs& g, int m_tiles, cudaStream_t st) {
+    constexpr int kChunks = kK / kKChunk;
+    constexpr int kStages = kChunks < kMaxStages ? kChunks : kMaxStages;
+    const size_t smem = (size_t)kStages * (kATile + (size_t)g.N * 128) + 8 * (2 * kStages + 1) + 16 + 1024;
+    if (cudaFuncSetAttribute(head_gemm_sm100_kernel<kK, kAMn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid(g.H, m_tiles, (g.R + g.N - 1) / g.N);
+    head_gemm_sm100_kernel<kK, kAMn><<<grid, kGemmThreads, smem, st>>>(g);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -149,25 +246,39 @@ extern "C" mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const
     using namespace mla;
     if (!q_nope || !q_rope || !w_uk || !q || R <= 0 || H <= 0) return MLA_ERR_INVALID_ARG;
     if (!aligned(q_nope, 16) || !aligned(w_uk, 16) || !aligned(q_rope, 16) || !aligned(q, 16)) return MLA_ERR_INVALID_ARG;
-    cudaStream_t st = (cudaStream_t)stream;
-    // X = q_nope [R, H, 128]; B_h = W_UK[h]^T: W_UK[h] is [512 x 128], contiguous along k
-    if (launch_head_gemm<true, 128, kDv>(reinterpret_cast<const __nv_bfloat16*>(q_nope), (int64_t)H * 128,
-                                         reinterpret_cast<const __nv_bfloat16*>(w_uk), reinterpret_cast<__nv_bfloat16*>(q),
-                                         (int64_t)H * kDqk, kDqk, R, H,
-                                         reinterpret_cast<const __nv_bfloat16*>(q_rope), st) != cudaSuccess)
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.N = n_tile(R);
+    // A = W_UK [H][512 d][128 k]: box of 64 k x 128 d of one head
+    if (!map_3d(&g.tm_a, w_uk, 128, kDv, (uint64_t)H, 128 * 2, (uint64_t)kDv * 128 * 2, 64, 128, 1)) return MLA_ERR_CUDA;
+    // X = q_nope [R][H][128 k]: box of 64 k x 1 head x N rows
+    if (!map_3d(&g.tm_x, q_nope, 128, (uint64_t)H, (uint64_t)R, 128 * 2, (uint64_t)H * 128 * 2, 64, 1, g.N))
         return MLA_ERR_CUDA;
-    return MLA_OK;
+    g.y = reinterpret_cast<__nv_bfloat16*>(q);
+    g.y_rs = (int64_t)H * kDqk;
+    g.y_hs = kDqk;
+    g.rope = reinterpret_cast<const __nv_bfloat16*>(q_rope);
+    g.R = R;
+    g.H = H;
+    return launch_head_gemm<128, false>(g, kDv / 128, (cudaStream_t)stream);
 }
 
 extern "C" mla_status mla_project_out(const void* out, const void* w_uv, int R, int H, void* y, void* stream) {
     using namespace mla;
     if (!out || !w_uv || !y || R <= 0 || H <= 0) return MLA_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(w_uv, 16) || !aligned(y, 4)) return MLA_ERR_INVALID_ARG;
-    // X = out [R, H, 512]; B_h = W_UV[h] [512 x 128], contiguous along n
-    return launch_head_gemm<false, kDv, 128>(reinterpret_cast<const __nv_bfloat16*>(out), (int64_t)H * kDv,
-                                             reinterpret_cast<const __nv_bfloat16*>(w_uv),
-                                             reinterpret_cast<__nv_bfloat16*>(y), (int64_t)H * 128, 128, R, H, nullptr,
-                                             (cudaStream_t)stream) == cudaSuccess
-               ? MLA_OK
-               : MLA_ERR_CUDA;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.N = n_tile(R);
+    // A = W_UV [H][512 d][128 c]: box of 64 c x 64 d of one head (MN-major atoms)
+    if (!map_3d(&g.tm_a, w_uv, 128, kDv, (uint64_t)H, 128 * 2, (uint64_t)kDv * 128 * 2, 64, 64, 1)) return MLA_ERR_CUDA;
+    // X = out [R][H][512 d]: box of 64 d x 1 head x N rows
+    if (!map_3d(&g.tm_x, out, kDv, (uint64_t)H, (uint64_t)R, kDv * 2, (uint64_t)H * kDv * 2, 64, 1, g.N))
+        return MLA_ERR_CUDA;
+    g.y = reinterpret_cast<__nv_bfloat16*>(y);
+    g.y_rs = (int64_t)H * 128;
+    g.y_hs = 128;
+    g.R = R;
+    g.H = H;
+    return launch_head_gemm<kDv, true>(g, 1, (cudaStream_t)stream);
 }

@@ -28,7 +28,10 @@ def _close_bf16(got, ref):
     assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 2e-3), float((err - 2.0 ** -8 * np.abs(ref)).max())
 
 
-@pytest.mark.parametrize("B,s_q,H", [(2, 4, 16), (16, 16, 16), (3, 1, 128), (1, 1, 1)])
+# R = B * s_q rows per head: 8, 256 (one full N tile), 3, 1, 64 x 128 heads (the fp8
+# workload), 15 (a ragged N tile), 320 (two N tiles)
+@pytest.mark.parametrize("B,s_q,H", [(2, 4, 16), (16, 16, 16), (3, 1, 128), (1, 1, 1), (32, 2, 128), (3, 5, 7),
+                                     (20, 16, 4)])
 def test_absorb_and_project_match_the_oracle(B, s_q, H):
     import torch
     rng = np.random.default_rng(B * 100 + H)
