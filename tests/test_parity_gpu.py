@@ -59,6 +59,19 @@ def test_edge_cases(kw, num_sms):
     _case("agent_spec", num_sms, **kw)
 
 
+@pytest.mark.parametrize("kw", [
+    dict(B=2, s_q=2, H=128, seq_lens=[2, 3]),                   # T = s_q: draft 0 sees one token
+    dict(B=9, s_q=1, H=64, seq_lens=[1, 2, 63, 64, 65, 127, 128, 129, 3000]),
+    dict(B=3, s_q=2, H=128, seq_lens=[64 * 3, 64 * 5 + 7, 64 * 2]),  # odd and even page counts
+    dict(B=2, s_q=4, H=48, seq_lens=[1500, 63]),                # M = 192: a partial third row block
+])
+@pytest.mark.parametrize("num_sms", [0, 4, 16])
+def test_edge_cases_e4m3(kw, num_sms):
+    """The e4m3 scan takes a split's pages in pairs: single-page units (odd counts, one-page
+    splits), pages exactly full and partial last pages, on plans of several shapes."""
+    _case("fp8_batch", num_sms, **kw)
+
+
 def test_many_short_requests():
     """More requests than the planner has threads: every planner loop makes several passes."""
     _case("agent_spec", 0, B=300, s_q=1, H=16, seq=("uniform", 1, 1500))
