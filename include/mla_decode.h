@@ -107,6 +107,10 @@ mla_status mla_decode_plan(const int32_t* seq_lens, int B, int s_q, int H, int n
  *   causal      != 0: draft i sees t <= T_b - s_q + i; 0: every t < T_b
  *   out         bf16 [B, s_q, H, 512];  lse  fp32 [B, s_q, H], natural log
  * Supported: s_q * H <= 256 per request.
+ * An e4m3 cache is read as it is by e4m3 x e4m3 tensor-core MMAs: q and the softmax
+ * weights P are each cut into two e4m3 terms (q at a per-row power-of-two scale, which
+ * holds a bf16 q exactly; P to 8 significant bits, as a bf16 P), so the results stay
+ * within the rounding of the bf16 path.
  */
 mla_status mla_decode(const void* q, const void* kv_pages, int kv_dtype, float kv_scale,
                       const int32_t* block_table, int max_pages_per_req,
@@ -152,8 +156,10 @@ mla_status mla_split_kv_combine(const void* workspace, size_t ws_bytes, int B, i
  * mla_project_out maps the decode's output to the heads' value space:
  *   y[r, h, :] = out[r, h, :] W_UV[h];  out bf16 [R, H, 512] and w_uv bf16 [H, 512, 128]
  *   (16-byte aligned), y bf16 [R, H, 128] (4-byte aligned).
- * Both accumulate in fp32 and round to bf16 (nearest, ties to even).  Argument errors
- * return before any launch.
+ * Both run on the tcgen05 tensor cores, accumulate in fp32 and round to bf16 (nearest,
+ * ties to even).  Argument errors return before any launch.  Every wait inside the kernel
+ * is bounded (2 s); these calls have no workspace and so no device status word: a wait
+ * that gave up (never expected) leaves its rows unwritten.
  */
 mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int R, int H, void* q,
                         void* stream);

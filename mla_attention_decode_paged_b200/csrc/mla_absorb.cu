@@ -47,7 +47,8 @@ struct __align__(64) GemmArgs {
     int64_t y_rs, y_hs;
     const __nv_bfloat16* rope;  // absorb only: q_rope [R, H, 64], copied to y[..., 512:576]
     int R, H, N;        // rows, heads, N tile (a multiple of 16, <= 256)
-    int32_t* status;    // where a bounded wait that gave up is recorded (may be null)
+    int32_t* status;    // where a bounded wait that gave up is recorded (null: these entry points have
+                        // no workspace; a wait that gives up leaves its rows unwritten)
 };
 
 // Bounded mbarrier wait (2 s); false if it gave up.
@@ -223,14 +224,25 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t
 // N tile: R rounded up to 16, at most 256 (the TMEM columns of one accumulator).
 int n_tile(int R) { return std::min(256, (R + 15) / 16 * 16); }
 
+template <int kK>
+constexpr size_t gemm_smem_bytes(int N) {
+    return (size_t)(kK / kKChunk < kMaxStages ? kK / kKChunk : kMaxStages) * (kATile + (size_t)N * 128) +
+           8 * (2 * kMaxStages + 1) + 16 + 1024;
+}
+
 template <int kK, bool kAMn>
 mla_status launch_head_gemm(const GemmArgs& g, int m_tiles, cudaStream_t st) {
-    constexpr int kChunks = kK / kKChunk;
-    constexpr int kStages = kChunks < kMaxStages ? kChunks : kMaxStages;
-    const size_t smem = (size_t)kStages * (kATile + (size_t)g.N * 128) + 8 * (2 * kStages + 1) + 16 + 1024;
-    if (cudaFuncSetAttribute(head_gemm_sm100_kernel<kK, kAMn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return MLA_ERR_CUDA;
+    // the shared memory opt-in, set once per device for the largest tile (N = 256)
+    static int done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev >= 64 || !done[dev]) {
+        if (cudaFuncSetAttribute(head_gemm_sm100_kernel<kK, kAMn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm_smem_bytes<kK>(256)) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (dev < 64) done[dev] = 1;
+    }
+    const size_t smem = gemm_smem_bytes<kK>(g.N);
     const dim3 grid(g.H, m_tiles, (g.R + g.N - 1) / g.N);
     head_gemm_sm100_kernel<kK, kAMn><<<grid, kGemmThreads, smem, st>>>(g);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
