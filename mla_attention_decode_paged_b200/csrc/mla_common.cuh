@@ -117,10 +117,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-    return __uint_as_float(((uint32_t)b) << 16);
-}
-
 // Two e4m3 bytes (low byte first) -> two floats, exact (every e4m3 value is an fp16 value).
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
     uint32_t h2;
