@@ -18,18 +18,21 @@ constexpr int kTileThreads = 256;     // 16 rows x 16 column quads
 constexpr int kWChunk = 64;           // splits whose weights are in shared memory at once
 constexpr int kPre = 6;               // partials per thread loaded before the weights are known
 
-// grid (B, 4 nqb, 8): one CTA per (request, 16-row group, 64 columns).  Within a group of
-// 256 threads, thread t owns row t % 16 and column quad t / 16 of the tile; in the
-// workspace's quad-interleaved partial layout the CTA's tile of one split is 4 KB
-// contiguous, read by the 256 threads with one 16-byte load each.  kSplitGroups groups
-// take the splits j = group, group + kSplitGroups, ... so that kSplitGroups x kPre
-// partials are in flight before the weights are known; the group sums meet in shared
-// memory at the end.  Four groups when requests have many splits (few long requests),
-// one when they have few (then more, smaller CTAs share an SM).
-template <int kSplitGroups>
+// One CTA per (request, 16-row group, kChunks column chunks of 64).  Within a group of
+// 256 threads, thread t owns row t % 16 and column quad t / 16 of a 16 x 64 tile; in the
+// workspace's quad-interleaved partial layout the tile of one split is 4 KB contiguous,
+// read by the 256 threads with one 16-byte load each.  kSplitGroups groups take the
+// splits j = group, group + kSplitGroups, ... so that kSplitGroups x kPre partials are in
+// flight before the weights are known; the group sums meet in shared memory at the end.
+// Four groups and one chunk per CTA when requests have many splits (few long requests:
+// enough CTAs, each with many partials); one group and all eight chunks when they have
+// few and there are at least 256 (request, 16-row group) pairs, so that the row weights
+// are computed once per 16 rows and the grid is one wave; two chunks for fewer pairs.
+template <int kSplitGroups, int kChunks>
 __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups) combine_kernel(
     const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     constexpr int kCombineThreads = kTileThreads * kSplitGroups;
+    static_assert(kSplitGroups == 1 || kChunks == 1, "split groups meet once per CTA");
     __shared__ float wsh[kWChunk][16];
     __shared__ float Lsh[16], Msh[16];
     __shared__ float4 part[kSplitGroups > 1 ? kSplitGroups - 1 : 1][kTileThreads];
@@ -37,7 +40,7 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     // launched as a programmatic dependent of the scan: nothing is read before it completes
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
-    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3, c64 = blockIdx.z;
+    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3;
     const int M = s_q * H;
     const int row0 = qb * kRowsPerBlock + g * 16;
     if (row0 >= M) return;
@@ -45,31 +48,40 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
     const int tid = threadIdx.x, t = tid & (kTileThreads - 1), grp = tid / kTileThreads;
     const int r16 = t & 15, cq = t >> 4;
+    const int m = row0 + r16;
     if (ns == 0) {
         // a request without tokens (T_b <= 0) has no split: the planner set the status word,
         // and its rows are written here as NaN
-        const int m = row0 + r16;
         if (grp == 0 && m < M) {
-            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
-                make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
-            if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
+#pragma unroll 1
+            for (int cc = 0; cc < kChunks; ++cc) {
+                const int c64 = blockIdx.z * kChunks + cc;
+                *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
+                    make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+            }
+            if (blockIdx.z == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
         }
         return;
     }
     if (ns == 1) return;  // written directly by the decode kernel
     const int nqb = h->nqb;
-    // split j: partial tile at pbase + j * jstride (float4), lse2 of row r at lbase[j * lstride + r]
+    // split j, column chunk c64: partial tile at pbase + c64 * 256 + j * jstride (float4),
+    // lse2 of row r at lbase[j * lstride + r]
     const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
-                          ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + (16 * c64 + cq) * 16 + r16;
+                          ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + cq * 16 + r16;
     const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
     const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
     const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
 
+    // the first chunk's partials, in flight while the weights are computed
     float4 v[kPre];
+    {
+        const float4* pc = pbase + (int64_t)(blockIdx.z * kChunks) * 256;
 #pragma unroll
-    for (int u = 0; u < kPre; ++u) {
-        const int j = grp + kSplitGroups * u;
-        v[u] = j < ns ? pbase[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < kPre; ++u) {
+            const int j = grp + kSplitGroups * u;
+            v[u] = j < ns ? pc[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
 
     // L = log2 sum_j 2^lse2_j per row: warp w < 8 takes rows 2w and 2w + 1 (one per half-warp)
@@ -99,61 +111,86 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
         }
     }
     __syncthreads();
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < ns; j0 += kWChunk) {
-        const int nj = min(kWChunk, ns - j0);
+    // the split weights 2^(lse2_j - L) of the 16 rows, for splits [j0, j0 + kWChunk)
+    auto weights = [&](int j0, int nj) {
         for (int e = tid; e < nj * 16; e += kCombineThreads) {
             const int jj = e >> 4, r = e & 15;
             const float l2 = lbase[(int64_t)(j0 + jj) * lstride + r];
             wsh[jj][r] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - Lsh[r]);  // an empty split drops out
         }
+    };
+    const bool one_wchunk = ns <= kWChunk;  // the weights of every split fit at once
+    if (one_wchunk) {
+        weights(0, ns);
         __syncthreads();
-        int jj = grp;  // this group's splits within the chunk: grp, grp + 4, ...
-        if (j0 == 0) {
+    }
+#pragma unroll 1
+    for (int cc = 0; cc < kChunks; ++cc) {
+        const int c64 = blockIdx.z * kChunks + cc;
+        const float4* pc = pbase + (int64_t)c64 * 256;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < ns; j0 += kWChunk) {
+            const int nj = min(kWChunk, ns - j0);
+            if (!one_wchunk) {
+                weights(j0, nj);
+                __syncthreads();
+            }
+            int jj = grp;  // this group's splits within the weight chunk: grp, grp + kSplitGroups, ...
+            if (j0 == 0) {
+#pragma unroll
+                for (int u = 0; u < kPre; ++u) {
+                    const int j = grp + kSplitGroups * u;
+                    const float w = j < nj ? wsh[j][r16] : 0.f;
+                    acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+                }
+                jj = grp + kSplitGroups * kPre;
+            }
+            for (; jj + kSplitGroups < nj; jj += 2 * kSplitGroups) {
+                float4 x[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) x[u] = pc[(j0 + jj + kSplitGroups * u) * jstride];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float w = wsh[jj + kSplitGroups * u][r16];
+                    acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
+                }
+            }
+            for (; jj < nj; jj += kSplitGroups) {
+                const float4 x = pc[(j0 + jj) * jstride];
+                const float w = wsh[jj][r16];
+                acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+            }
+            if (!one_wchunk) __syncthreads();
+        }
+        // the next chunk's first partials, in flight while this chunk is finished
+        if (cc + 1 < kChunks) {
+            const float4* pn = pc + 256;
 #pragma unroll
             for (int u = 0; u < kPre; ++u) {
                 const int j = grp + kSplitGroups * u;
-                const float w = j < nj ? wsh[j][r16] : 0.f;
-                acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
-            }
-            jj = grp + kSplitGroups * kPre;
-        }
-        for (; jj + kSplitGroups < nj; jj += 2 * kSplitGroups) {
-            float4 x[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) x[u] = pbase[(j0 + jj + kSplitGroups * u) * jstride];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const float w = wsh[jj + kSplitGroups * u][r16];
-                acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
+                v[u] = j < ns ? pn[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        for (; jj < nj; jj += kSplitGroups) {
-            const float4 x = pbase[(j0 + jj) * jstride];
-            const float w = wsh[jj][r16];
-            acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
-        }
-        __syncthreads();
-    }
-    if (kSplitGroups > 1) {
-        if (grp > 0) part[grp - 1][t] = acc;
-        __syncthreads();
-        if (grp > 0) return;
+        if (kSplitGroups > 1) {
+            // (one chunk per CTA here: the groups' sums meet once, then the other groups leave)
+            if (grp > 0) part[grp - 1][t] = acc;
+            __syncthreads();
+            if (grp > 0) return;
 #pragma unroll
-        for (int k = 0; k < kSplitGroups - 1; ++k) {
-            const float4 x = part[k][t];
-            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            for (int k = 0; k < kSplitGroups - 1; ++k) {
+                const float4 x = part[k][t];
+                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            }
         }
-    }
-    const int m = row0 + r16;
-    if (m < M) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) = pk;
-        if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
+        if (grp == 0 && m < M) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) = pk;
+            if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
+        }
     }
 }
 
@@ -163,9 +200,13 @@ mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, floa
     const int sms = effective_sms();
     const int G = num_groups_for(sms > 0 ? sms : 1, num_row_blocks(s_q, H));
     const bool many_splits = (int64_t)B + G >= 8 * (int64_t)B;
+    // with few splits a CTA takes all eight column chunks of its 16 rows when that still
+    // leaves enough CTAs (the row weights are then computed once), else two
+    const int64_t row_groups = (int64_t)B * 4 * num_row_blocks(s_q, H);
+    const int chunks = many_splits ? 1 : (row_groups >= 256 ? 8 : 2);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(B, 4 * num_row_blocks(s_q, H), kDv / 64);
+    cfg.gridDim = dim3(B, 4 * num_row_blocks(s_q, H), (kDv / 64) / chunks);
     cfg.blockDim = dim3(kTileThreads * (many_splits ? 4 : 1));
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -174,8 +215,9 @@ mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, floa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-    const cudaError_t e = many_splits ? cudaLaunchKernelEx(&cfg, combine_kernel<4>, ws, B, s_q, H, o, lse)
-                                      : cudaLaunchKernelEx(&cfg, combine_kernel<1>, ws, B, s_q, H, o, lse);
+    const cudaError_t e = chunks == 1   ? cudaLaunchKernelEx(&cfg, combine_kernel<4, 1>, ws, B, s_q, H, o, lse)
+                          : chunks == 8 ? cudaLaunchKernelEx(&cfg, combine_kernel<1, 8>, ws, B, s_q, H, o, lse)
+                                        : cudaLaunchKernelEx(&cfg, combine_kernel<1, 2>, ws, B, s_q, H, o, lse);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
