@@ -16,42 +16,39 @@
 namespace mla {
 
 constexpr int kPlanThreads = 256;
+constexpr int kPlanWarps = kPlanThreads / 32;
+static_assert(kPlanWarps == 8, "plan_shared_bytes reserves 8 words of scan scratch");
 
-// In-place exclusive prefix sum of a[0..n) by the whole block (n + 1 entries are written:
-// a[n] receives the total).  Each thread scans a contiguous chunk; the chunk totals are
-// scanned with warp shuffles (one warp per 32 chunks, then one warp over the 8 warp sums).
-// The caller synchronises the block before the call; the call ends with a barrier.  Not
-// inlined: the plan runs once per launch on a cold SM, so one shared copy of the code
-// costs fewer instruction fetches than three inlined ones.
-__device__ __noinline__ void block_exclusive_scan(int64_t* a, int n, int64_t* partial) {
-    static_assert(kPlanThreads == 256, "two-level warp scan below assumes 8 warps");
+// Thread t's contiguous share [x, y) of n items: the loads, the flag tests and the scans
+// below give every thread the same share, so a thread scans only what it wrote itself
+// and no barrier is needed between writing an array and scanning it.
+__device__ __forceinline__ int2 chunk_of(int n) {
     const int per = (n + kPlanThreads - 1) / kPlanThreads;
-    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    const int lo = min(n, (int)threadIdx.x * per);
+    return make_int2(lo, min(n, lo + per));
+}
+
+// In-place exclusive prefix sum of a[0..n) by the whole block; a[n] receives the total.
+// Each thread scans its own chunk; chunk totals are scanned with warp shuffles and the
+// warp totals are added by every thread from shared memory.  Two barriers, the second
+// ends the call.
+__device__ __forceinline__ void block_exclusive_scan(int64_t* a, int n, int64_t* wsum) {
+    const int2 c = chunk_of(n);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int64_t run = 0;
-    for (int i = lo; i < hi; ++i) run += a[i];
-    // inclusive scan of the chunk totals within the warp
+    for (int i = c.x; i < c.y; ++i) run += a[i];
     int64_t v = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int64_t u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
     }
-    if (lane == 31) partial[warp] = v;
+    if (lane == 31) wsum[warp] = v;
     __syncthreads();
-    if (warp == 0) {
-        int64_t w = lane < 8 ? partial[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            const int64_t u = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += u;
-        }
-        if (lane < 8) partial[8 + lane] = w;  // inclusive totals of warps 0..lane
-    }
-    __syncthreads();
-    int64_t acc = (v - run) + (warp > 0 ? partial[8 + warp - 1] : 0);  // exclusive offset of this chunk
-    if (threadIdx.x == kPlanThreads - 1) a[n] = partial[15];
-    for (int i = lo; i < hi; ++i) {
+    int64_t acc = v - run;  // exclusive offset of this chunk
+    for (int w = 0; w < warp; ++w) acc += wsum[w];
+    if (threadIdx.x == kPlanThreads - 1) a[n] = acc + run;
+    for (int i = c.x; i < c.y; ++i) {
         const int64_t x = a[i];
         a[i] = acc;
         acc += x;
@@ -59,33 +56,39 @@ __device__ __noinline__ void block_exclusive_scan(int64_t* a, int n, int64_t* pa
     __syncthreads();
 }
 
-// first index i in [0, n) with a[i] >= x (a non-decreasing), n if none
-__device__ __noinline__ int lower_bound64(const int64_t* a, int n, int64_t x) {
-    int lo = 0, hi = n;
+// last request index b in [0, B] whose first page is <= x (pk: pages before b in the
+// high word, non-decreasing); x >= 0
+__device__ __forceinline__ int last_start_le(const int64_t* pk, int B, int64_t x) {
+    const int64_t key = (x + 1) << 32;
+    int lo = 0, hi = B + 1;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (a[mid] < x) lo = mid + 1; else hi = mid;
+        if (pk[mid] < key) lo = mid + 1; else hi = mid;
     }
-    return lo;
+    return lo - 1;
 }
 
-// One CTA, everything in shared memory and in parallel:
-//   pk[b]    (pages before request b) << 32 | (requests with tokens before b): one scan of
+// One CTA, everything in shared memory:
+//   pk[b]    (pages before request b) << 32 | (requests with pages before b): one scan of
 //            (ceil(T_b / 64) << 32 | [T_b > 0]); the low field never carries into the high one;
-//   cut(g)   share boundary floor(total * g / G), and the first g whose cut is >= x in
-//            closed form, ceil(x * G / total);
+//   cut[g]   share boundary floor(total * g / G);
 //   a cut that falls strictly inside a request, and is the first of its value, starts a new
-//   segment ("flagged"); every request with pages starts one;
-//   a request's segments are its start plus its flagged cuts; a group's first segment is
-//   the number of segment starts below its boundary.
+//   segment ("flagged"); every request with pages starts one.  Segments are numbered in
+//   page order, so a segment's index is the number of segment starts below it: requests
+//   with pages that start below it plus flagged cuts below it.  Each start is recorded at
+//   its index; a segment ends where the next one of its request starts, or at the
+//   request's end.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ seq_lens, int B, int s_q,
                                                             int H, WsLayout L, void* ws) {
     const int G = L.num_groups;
     extern __shared__ int64_t plan_sh[];
-    int64_t* pk = plan_sh;             // [B + 1]
-    int64_t* flag = pk + (B + 1);      // [G + 2] -> flagged cuts before g
-    int64_t* nseg = flag + (G + 2);    // [B + 1] -> first segment of request b
-    int64_t* part = nseg + (B + 1);    // [16] scan scratch
+    int64_t* pk = plan_sh;                                        // [B + 1]
+    int64_t* cut = pk + (B + 1);                                  // [G + 1]
+    int64_t* fsum = cut + (G + 1);                                // [G + 2] flags, then flagged cuts below g
+    int64_t* wsum = fsum + (G + 2);                               // [kPlanWarps] scan scratch
+    int32_t* inside = reinterpret_cast<int32_t*>(wsum + kPlanWarps);  // [G + 1] request a flagged cut cuts
+    int32_t* rec_b = inside + (G + 1);                            // [B + G] segment starts: request
+    int32_t* rec_t = rec_b + (B + G);                             // [B + G] segment starts: first page in it
     __shared__ int bad_first;
     PlanHeader* h = reinterpret_cast<PlanHeader*>(ws);
     int32_t* group_begin = ws_ptr<int32_t>(ws, L.off_group_begin);
@@ -96,80 +99,68 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     // grid to complete before reading the plan
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    if (tid == 0) bad_first = B;
-    __syncthreads();
-    for (int b = tid; b < B; b += kPlanThreads) {
-        const int T = seq_lens[b];
-        pk[b] = T > 0 ? ((int64_t)((T + kPage - 1) / kPage) << 32) | 1 : 0;
-        if (T <= 0) atomicMin(&bad_first, b);
+    if (tid == 0) bad_first = -1;
+    {
+        const int2 c = chunk_of(B);
+        for (int b = c.x; b < c.y; ++b) {
+            const int64_t T = seq_lens[b];
+            pk[b] = T > 0 ? ((T + kPage - 1) / kPage) << 32 | 1 : 0;
+        }
     }
-    __syncthreads();
-    block_exclusive_scan(pk, B, part);
+    block_exclusive_scan(pk, B, wsum);
     const int64_t total = pk[B] >> 32;
-    // first g in [0, G] with cut(g) >= x; G + 1 if none
+    const int nvalid = (int)(pk[B] & 0xffffffff);
+    {
+        const int2 c = chunk_of(G + 1);
+        for (int g = c.x; g < c.y; ++g) {
+            const int64_t cg = total * g / G;
+            int64_t f = 0;
+            int in = -1;
+            if (g > 0 && g < G && cg > 0 && cg < total && cg != total * (g - 1) / G) {
+                // the last request starting at or below cg starts exactly there (and has
+                // pages), or cg falls strictly inside it
+                const int bl = last_start_le(pk, B, cg);
+                if ((pk[bl] >> 32) != cg) {
+                    f = 1;
+                    in = bl;
+                }
+            }
+            cut[g] = cg;
+            fsum[g] = f;
+            inside[g] = in;
+        }
+    }
+    block_exclusive_scan(fsum, G + 1, wsum);  // fsum[g] = flagged cuts with index < g
+    const int nseg_total = nvalid + (int)fsum[G + 1];
+    // first g in [0, G] with cut[g] >= x, i.e. ceil(x * G / total); G + 1 if none.  A float
+    // estimate, corrected against the exact cuts.
     auto first_cut_ge = [&](int64_t x) -> int {
         if (x <= 0) return 0;
         if (x > total) return G + 1;
-        return (int)((x * G + total - 1) / total);
+        int g = (int)ceilf((float)x * (float)G / (float)total);
+        g = min(max(g, 0), G);
+        while (g > 0 && cut[g - 1] >= x) --g;
+        while (g < G && cut[g] < x) ++g;
+        return g;
     };
-    for (int g = tid; g <= G; g += kPlanThreads) {
-        int64_t f = 0;
-        if (g > 0 && g < G) {
-            const int64_t cg = total * g / G;
-            if (cg > 0 && cg < total && cg != total * (g - 1) / G) {
-                // a request start? the last request whose start is <= cg starts exactly at cg
-                // and has pages
-                const int bl = lower_bound64(pk, B + 1, (cg + 1) << 32) - 1;
-                const bool is_start = bl < B && (pk[bl] >> 32) == cg && (pk[bl + 1] >> 32) > cg;
-                f = is_start ? 0 : 1;
-            }
-        }
-        flag[g] = f;
-    }
-    __syncthreads();
-    block_exclusive_scan(flag, G + 1, part);  // flag[g] = flagged cuts with index < g
     for (int b = tid; b < B; b += kPlanThreads) {
         const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
-        int64_t n = 0;
+        const int before = (int)(pk[b] & 0xffffffff);
+        const int first = before + (int)fsum[first_cut_ge(p0)];
+        req_seg[b] = first;
         if (p1 > p0) {
-            const int gl = first_cut_ge(p0 + 1), gh = first_cut_ge(p1);
-            n = 1 + (gh > gl ? flag[gh] - flag[gl] : 0);
+            rec_b[first] = b;
+            rec_t[first] = 0;
+        } else if (before == b) {
+            bad_first = b;  // the first request without tokens: every one before it has some
         }
-        nseg[b] = n;
-    }
-    __syncthreads();
-    block_exclusive_scan(nseg, B, part);  // nseg[b] = first segment of request b
-    const int nseg_total = (int)nseg[B];
-    // segments, in parallel: every request with pages starts its first segment at tile 0,
-    // every flagged cut starts the next segment of the request it falls in; a segment ends
-    // at the next flagged cut inside its request (found by a search of the scanned flags:
-    // cut g is flagged iff flag[g + 1] > flag[g]) or at the request's end
-    for (int b = tid; b < B; b += kPlanThreads) {
-        req_seg[b] = (int)nseg[b];
-        const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
-        if (p1 <= p0) continue;
-        const int gl = first_cut_ge(p0 + 1), gh = first_cut_ge(p1);
-        const int g1 = lower_bound64(flag, G + 2, flag[gl] + 1) - 1;  // first flagged cut >= gl
-        Segment sg;
-        sg.b = b;
-        sg.tile_begin = 0;
-        sg.tile_end = (int32_t)((g1 < gh ? total * g1 / G : p1) - p0);
-        sg.split = nseg[b + 1] - nseg[b] > 1;
-        segs[nseg[b]] = sg;
     }
     for (int g = tid + 1; g < G; g += kPlanThreads) {
-        if (flag[g + 1] == flag[g]) continue;  // not a flagged cut
-        const int64_t cg = total * g / G;
-        const int b = lower_bound64(pk, B + 1, (cg + 1) << 32) - 1;  // the request cg falls strictly inside
-        const int64_t p0 = pk[b] >> 32, p1 = pk[b + 1] >> 32;
-        const int gh = first_cut_ge(p1);
-        const int g2 = lower_bound64(flag, G + 2, flag[g + 1] + 1) - 1;  // next flagged cut after g
-        Segment sg;
-        sg.b = b;
-        sg.tile_begin = (int32_t)(cg - p0);
-        sg.tile_end = (int32_t)((g2 < gh ? total * g2 / G : p1) - p0);
-        sg.split = 1;
-        segs[nseg[b] + 1 + (flag[g] - flag[first_cut_ge(p0 + 1)])] = sg;
+        const int b = inside[g];
+        if (b < 0) continue;
+        const int idx = (int)(pk[b] & 0xffffffff) + 1 + (int)fsum[g];
+        rec_b[idx] = b;
+        rec_t[idx] = (int32_t)(cut[g] - (pk[b] >> 32));
     }
     for (int g = tid; g <= G; g += kPlanThreads) {
         int v;
@@ -178,16 +169,29 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         } else if (g == G) {
             v = nseg_total;
         } else {
-            // segment starts below cut(g): request starts below it plus flagged cuts below it
-            const int64_t x = total * g / G;
-            const int bx = lower_bound64(pk, B, x << 32);  // requests 0..bx-1 start below x
-            v = (int)(pk[bx] & 0xffffffff) + (int)flag[first_cut_ge(x)];
+            // segment starts below cut(g): requests with pages starting below it plus
+            // flagged cuts below it
+            const int64_t x = cut[g];
+            const int bl = last_start_le(pk, B, x);
+            const int below = (int)(((pk[bl] >> 32) == x ? pk[bl] : pk[bl + 1]) & 0xffffffff);
+            v = below + (int)fsum[first_cut_ge(x)];
         }
         group_begin[g] = v;
     }
+    __syncthreads();
+    for (int i = tid; i < nseg_total; i += kPlanThreads) {
+        const int b = rec_b[i];
+        const bool last = i + 1 == nseg_total || rec_b[i + 1] != b;
+        Segment sg;
+        sg.b = b;
+        sg.tile_begin = rec_t[i];
+        sg.tile_end = last ? (int32_t)((pk[b + 1] >> 32) - (pk[b] >> 32)) : rec_t[i + 1];
+        sg.split = !(last && rec_t[i] == 0);
+        segs[i] = sg;
+    }
     if (tid == 0) {
         req_seg[B] = nseg_total;
-        const int bad = bad_first < B ? bad_first : -1;
+        const int bad = bad_first;
         h->status = bad >= 0 ? kStatusOob : kStatusOk;
         h->status_info = bad >= 0 ? bad : 0;
         h->B = B;

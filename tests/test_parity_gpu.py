@@ -121,7 +121,14 @@ def test_page_permutation_leaves_the_result_within_rounding():
 @pytest.mark.parametrize("lens,s_q,H,num_sms", [([65536] * 4, 4, 16, 148), ([70000, 1, 64, 65, 30000], 2, 128, 148),
                                                 ([300] * 3, 8, 32, 8), ([5] * 7, 1, 16, 1),
                                                 (list(np.random.default_rng(1).integers(1, 3000, 600)), 1, 16, 148),
-                                                ([0, 100, 0, 5000], 1, 16, 148)])
+                                                ([0, 100, 0, 5000], 1, 16, 148),
+                                                # more groups than pages: runs of equal cuts
+                                                ([1, 1, 1], 1, 16, 1023), ([64] * 3 + [0] * 5 + [65], 4, 16, 1000),
+                                                # several thousand requests (several per planner thread), some empty
+                                                (list(np.where(np.random.default_rng(2).random(5000) < 0.1, 0,
+                                                               np.random.default_rng(3).integers(1, 4000, 5000))),
+                                                 1, 16, 148),
+                                                ([-5, 10, 0], 2, 16, 148), ([131072] * 16, 16, 16, 148)])
 def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     import torch
     import mla_attention_decode_paged_b200 as mla
@@ -134,6 +141,8 @@ def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     egb, ers, esegs = plan_ref.plan(lens, G)
     assert h32[2] == 0x4D4C4131 and h32[7] == G
     assert np.array_equal(gb, egb) and np.array_equal(rs, ers) and np.array_equal(segs, esegs)
+    bad = [b for b, t in enumerate(lens) if t <= 0]  # a request without tokens is reported, the first one
+    assert (h32[0], h32[1]) == ((5, bad[0]) if bad else (0, 0))
 
 
 def test_bad_page_id_sets_device_status_and_poisons_only_that_request():
