@@ -55,8 +55,19 @@ struct __align__(16) PlanHeader {
     int64_t total_bytes;
 };
 
+// A group's segment range and its first segment, at a fixed place in the workspace
+// (kOffHeads + 32 g): a scan CTA reads it together with the plan header, so that its first
+// page loads wait for one round trip to memory instead of three.
+struct __align__(16) GroupHead {
+    int32_t seg_lo, seg_hi;  // the group's segments [seg_lo, seg_hi)
+    int32_t pad0, pad1;
+    Segment first;           // segment seg_lo (zeros for a group without pages)
+};
+constexpr int64_t kOffHeads = 256;
+static_assert(sizeof(PlanHeader) <= kOffHeads, "the head table follows the header");
+
 struct WsLayout {
-    int64_t off_group_begin, off_req_seg, off_segs, off_plse, off_po, total;
+    int64_t off_heads, off_group_begin, off_req_seg, off_segs, off_plse, off_po, total;
     int nqb, num_groups, max_segments;
 };
 
@@ -79,7 +90,9 @@ __host__ __device__ inline WsLayout make_layout(int B, int s_q, int H, int num_g
     L.nqb = num_row_blocks(s_q, H);
     L.num_groups = num_groups;
     L.max_segments = B + num_groups;
-    int64_t o = align_up((int64_t)sizeof(PlanHeader), 256);
+    int64_t o = kOffHeads;
+    L.off_heads = o;
+    o = align_up(o + (int64_t)sizeof(GroupHead) * num_groups, 256);
     L.off_group_begin = o;
     o = align_up(o + 4 * (int64_t)(num_groups + 1), 256);
     L.off_req_seg = o;

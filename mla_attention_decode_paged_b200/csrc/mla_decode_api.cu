@@ -40,6 +40,10 @@ extern "C" mla_status mla_decode_scan(const void* q, const void* kv_pages, int k
     p.M = s_q * H;
     p.causal = causal != 0;
     p.groups_launched = num_groups_for(sms, num_row_blocks(s_q, H));
+    // the scan reads its group's head record before it checks the plan (always true for a
+    // workspace of at least one group's layout; kept explicit)
+    if ((int64_t)ws_bytes < kOffHeads + (int64_t)sizeof(GroupHead) * p.groups_launched)
+        return MLA_ERR_WORKSPACE_TOO_SMALL;
     const float ks = kv_dtype == MLA_KV_E4M3 ? kv_scale : 1.f;
     p.score_scale_log2 = scale * ks * kLog2e;
     p.out_scale = ks;

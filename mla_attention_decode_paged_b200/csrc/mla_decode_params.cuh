@@ -28,8 +28,9 @@ struct DecodeParams {
 inline size_t plan_shared_bytes(int B, int G) {
     const size_t b = (size_t)B, g = (size_t)G;
     // int64: prefix over requests [B + 1], cuts [G + 1], flags [G + 2], scan scratch [8];
-    // int32: the request each cut falls inside [G + 1], segment starts 2 x [B + G]
-    return sizeof(int64_t) * ((b + 1) + (g + 1) + (g + 2) + 8) + sizeof(int32_t) * ((g + 1) + 2 * (b + g));
+    // int32: the request each cut falls inside [G + 1], segment starts 2 x [B + G], first
+    // segment of each group [G + 1]
+    return sizeof(int64_t) * ((b + 1) + (g + 1) + (g + 2) + 8) + sizeof(int32_t) * (2 * (g + 1) + 2 * (b + g));
 }
 constexpr size_t kPlanMaxSharedBytes = 200 * 1024;
 

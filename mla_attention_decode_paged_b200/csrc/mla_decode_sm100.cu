@@ -120,10 +120,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
 
     // the plan (and every earlier write) must be complete before the header is read
     ptx::griddep_wait();
+    // The header and this group's head record are read together: the head table sits at a
+    // fixed offset, and every workspace the host accepts holds it for any group launched.
+    const int nqb = num_row_blocks(p.s_q, p.H);
+    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
+    const GroupHead gh = ws_ptr<GroupHead>(p.ws, kOffHeads)[g];
     const bool plan_ok = h->magic == kPlanMagic && h->B == p.B && h->s_q == p.s_q && h->H == p.H &&
                          h->num_groups <= p.groups_launched;
-    const int nqb = plan_ok ? h->nqb : 1;
-    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
     if (!plan_ok || g >= h->num_groups) {
         if (!plan_ok && blockIdx.x == 0 && threadIdx.x == 0) set_status(h, kStatusPlanMismatch, 0);
         ptx::tc_fence_before();
@@ -133,9 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         return;
     }
 
-    const int32_t* group_begin = ws_ptr<int32_t>(p.ws, h->off_group_begin);
     const Segment* segs = ws_ptr<Segment>(p.ws, h->off_segs);
-    const int seg_lo = group_begin[g], seg_hi = group_begin[g + 1];
+    const int seg_lo = gh.seg_lo, seg_hi = gh.seg_hi;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -146,15 +148,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         bool ok = true;
         for (int si = seg_lo; si < seg_hi && ok; ++si) {
             if (__shfl_sync(0xffffffffu, lane == 0 ? *c.abort : 0, 0)) break;
-            const Segment S = segs[si];
+            const Segment S = si == seg_lo ? gh.first : segs[si];
+            const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
+            // the first window of page ids is read beside the length (both wait on the same
+            // round trip); a window slot past max_pages is never read
+            const int t_first = S.tile_begin + lane;
+            const int32_t pg_first = (t_first < S.tile_end && t_first < p.max_pages) ? bt_row[t_first] : 0;
             const int T = p.seq_lens[S.b];
             if (!request_ok(p, T)) continue;
-            const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
             int32_t pg = 0, pgn = 0;  // page ids of tiles [t0, t0 + 32) and [t0 + 32, t0 + 64)
             for (int t = S.tile_begin; t < S.tile_end; ++t, ++it) {
                 const int j = (t - S.tile_begin) & 31;
                 if (j == 0) {
-                    pg = t == S.tile_begin ? ((t + lane < S.tile_end) ? bt_row[t + lane] : 0) : pgn;
+                    pg = t == S.tile_begin ? pg_first : pgn;
                     pgn = (t + 32 + lane < S.tile_end) ? bt_row[t + 32 + lane] : 0;
                 }
                 const int32_t page = __shfl_sync(0xffffffffu, pg, j);
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
             int it = 0, nseg = 0;
             bool ok = true;
             for (int si = seg_lo; si < seg_hi && ok; ++si) {
-                const Segment S = segs[si];
+                const Segment S = si == seg_lo ? gh.first : segs[si];
                 const int T = p.seq_lens[S.b];
                 if (!request_ok(p, T)) continue;
                 if (!wait_bar(c, c.bar(B_Q_FULL), nseg & 1)) break;
@@ -280,26 +286,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         bool alive = true;
 
         for (int si = seg_lo; si < seg_hi; ++si) {
-            const Segment S = segs[si];
+            const Segment S = si == seg_lo ? gh.first : segs[si];
             const int T = p.seq_lens[S.b];
+            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row.
+            // The loads are all issued before the first is used, beside the length's read: at a
+            // split's start the memory system is full of the first pages' loads, and every
+            // dependent round trip here delays the first score MMA.
+            const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + r.m_glob) * kDqk);
+            uint4 x[9][4];
+#pragma unroll
+            for (int k = 0; k < 9; ++k)
+#pragma unroll
+                for (int w = 0; w < 4; ++w)  // dims [64 k + 32 half, +32)
+                    x[k][w] = r.row_valid ? src[(64 * k + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
             if (!request_ok(p, T)) {
                 if (tid == 0) set_status(h, kStatusOob, S.b);
                 poison_rows(p, S, si, r, po, plse);
                 continue;
             }
             if (*c.abort) break;
-            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row.
-            // The loads are all issued before the first is used: at a split's start the memory
-            // system is full of the first pages' loads, and every dependent round trip here
-            // delays the first score MMA.
             {
-                const uint4* src = reinterpret_cast<const uint4*>(qsrc + ((int64_t)S.b * p.M + r.m_glob) * kDqk);
-                uint4 x[9][4];
-#pragma unroll
-                for (int k = 0; k < 9; ++k)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)  // dims [64 k + 32 half, +32)
-                        x[k][w] = r.row_valid ? src[(64 * k + 32 * half) / 8 + w] : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int k = 0; k < 9; ++k) {
                     uint32_t v[16];

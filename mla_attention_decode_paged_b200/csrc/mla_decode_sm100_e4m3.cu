@@ -140,10 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
 
     // the plan (and every earlier write) must be complete before the header is read
     ptx::griddep_wait();
+    // The header and this group's head record are read together: the head table sits at a
+    // fixed offset, and every workspace the host accepts holds it for any group launched.
+    const int nqb = num_row_blocks(p.s_q, p.H);
+    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
+    const GroupHead gh = ws_ptr<GroupHead>(p.ws, kOffHeads)[g];
     const bool plan_ok = h->magic == kPlanMagic && h->B == p.B && h->s_q == p.s_q && h->H == p.H &&
                          h->num_groups <= p.groups_launched;
-    const int nqb = plan_ok ? h->nqb : 1;
-    const int g = blockIdx.x / nqb, qb = blockIdx.x % nqb;
     if (!plan_ok || g >= h->num_groups) {
         if (!plan_ok && blockIdx.x == 0 && threadIdx.x == 0) set_status(h, kStatusPlanMismatch, 0);
         ptx::tc_fence_before();
@@ -153,9 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
         return;
     }
 
-    const int32_t* group_begin = ws_ptr<int32_t>(p.ws, h->off_group_begin);
     const Segment* segs = ws_ptr<Segment>(p.ws, h->off_segs);
-    const int seg_lo = group_begin[g], seg_hi = group_begin[g + 1];
+    const int seg_lo = gh.seg_lo, seg_hi = gh.seg_hi;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -166,16 +168,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
         bool ok = true;
         for (int si = seg_lo; si < seg_hi && ok; ++si) {
             if (__shfl_sync(0xffffffffu, lane == 0 ? *c.abort : 0, 0)) break;
-            const Segment S = segs[si];
+            const Segment S = si == seg_lo ? gh.first : segs[si];
+            const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
+            // the first window of page ids is read beside the length (both wait on the same
+            // round trip); a window slot past max_pages is never read
+            const int t_first = S.tile_begin + lane;
+            const int32_t pg_first = (t_first < S.tile_end && t_first < p.max_pages) ? bt_row[t_first] : 0;
             const int T = p.seq_lens[S.b];
             if (!request_ok(p, T)) continue;
-            const int32_t* bt_row = p.block_table + (int64_t)S.b * p.max_pages;
             const int n = S.tile_end - S.tile_begin;
             int32_t pg = 0, pgn = 0;  // page ids of tiles [t0, t0 + 32) and [t0 + 32, t0 + 64)
             for (int t = S.tile_begin; t < S.tile_end; ++t) {
                 const int jt = t - S.tile_begin, j = jt & 31, w = jt & 1;
                 if (j == 0) {
-                    pg = t == S.tile_begin ? ((t + lane < S.tile_end) ? bt_row[t + lane] : 0) : pgn;
+                    pg = t == S.tile_begin ? pg_first : pgn;
                     pgn = (t + 32 + lane < S.tile_end) ? bt_row[t + 32 + lane] : 0;
                 }
                 const int32_t page = __shfl_sync(0xffffffffu, pg, j);
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
             int un = 0, nseg = 0;
             bool ok = true;
             for (int si = seg_lo; si < seg_hi && ok; ++si) {
-                const Segment S = segs[si];
+                const Segment S = si == seg_lo ? gh.first : segs[si];
                 const int T = p.seq_lens[S.b];
                 if (!request_ok(p, T)) continue;
                 if (!wait_bar(c, c.bar(B_Q_FULL), nseg & 1)) break;
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
         bool alive = true;
 
         for (int si = seg_lo; si < seg_hi; ++si) {
-            const Segment S = segs[si];
+            const Segment S = si == seg_lo ? gh.first : segs[si];
             const int T = p.seq_lens[S.b];
             if (!request_ok(p, T)) {
                 if (tid == 0) set_status(h, kStatusOob, S.b);

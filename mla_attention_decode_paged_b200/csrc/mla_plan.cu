@@ -89,9 +89,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     int32_t* inside = reinterpret_cast<int32_t*>(wsum + kPlanWarps);  // [G + 1] request a flagged cut cuts
     int32_t* rec_b = inside + (G + 1);                            // [B + G] segment starts: request
     int32_t* rec_t = rec_b + (B + G);                             // [B + G] segment starts: first page in it
+    int32_t* gb_s = rec_t + (B + G);                              // [G + 1] first segment of each group
     __shared__ int bad_first;
     PlanHeader* h = reinterpret_cast<PlanHeader*>(ws);
     int32_t* group_begin = ws_ptr<int32_t>(ws, L.off_group_begin);
+    GroupHead* heads = ws_ptr<GroupHead>(ws, L.off_heads);
     int32_t* req_seg = ws_ptr<int32_t>(ws, L.off_req_seg);
     Segment* segs = ws_ptr<Segment>(ws, L.off_segs);
     const int tid = threadIdx.x;
@@ -177,9 +179,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
             v = below + (int)fsum[first_cut_ge(x)];
         }
         group_begin[g] = v;
+        gb_s[g] = v;
     }
     __syncthreads();
-    for (int i = tid; i < nseg_total; i += kPlanThreads) {
+    auto segment_at = [&](int i) -> Segment {
         const int b = rec_b[i];
         const bool last = i + 1 == nseg_total || rec_b[i + 1] != b;
         Segment sg;
@@ -187,7 +190,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         sg.tile_begin = rec_t[i];
         sg.tile_end = last ? (int32_t)((pk[b + 1] >> 32) - (pk[b] >> 32)) : rec_t[i + 1];
         sg.split = !(last && rec_t[i] == 0);
-        segs[i] = sg;
+        return sg;
+    };
+    for (int i = tid; i < nseg_total; i += kPlanThreads) segs[i] = segment_at(i);
+    for (int g = tid; g < G; g += kPlanThreads) {
+        GroupHead gh;
+        gh.seg_lo = gb_s[g];
+        gh.seg_hi = gb_s[g + 1];
+        gh.pad0 = gh.pad1 = 0;
+        if (gh.seg_lo < gh.seg_hi) {
+            gh.first = segment_at(gh.seg_lo);
+        } else {
+            gh.first.b = gh.first.tile_begin = gh.first.tile_end = gh.first.split = 0;
+        }
+        heads[g] = gh;
     }
     if (tid == 0) {
         req_seg[B] = nseg_total;

@@ -143,6 +143,13 @@ def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     assert np.array_equal(gb, egb) and np.array_equal(rs, ers) and np.array_equal(segs, esegs)
     bad = [b for b, t in enumerate(lens) if t <= 0]  # a request without tokens is reported, the first one
     assert (h32[0], h32[1]) == ((5, bad[0]) if bad else (0, 0))
+    # each group's head record (read by the scan beside the header): its segment range and
+    # a copy of its first segment
+    heads = ws.cpu().numpy()[256:256 + 32 * G].view(np.int32).reshape(G, 8)
+    assert np.array_equal(heads[:, 0], egb[:-1]) and np.array_equal(heads[:, 1], egb[1:])
+    for g in range(G):
+        want = esegs[egb[g]] if egb[g] < egb[g + 1] else np.zeros(4, np.int32)
+        assert np.array_equal(heads[g, 4:], want), g
 
 
 def test_bad_page_id_sets_device_status_and_poisons_only_that_request():
