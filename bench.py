@@ -54,7 +54,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # B200 datasheet (dense bf16), for context
 KERNEL_SOURCES = ["mla_attention_decode_paged_b200/csrc/mla_decode_sm100.cu",
                   "mla_attention_decode_paged_b200/csrc/mla_decode_sm100_e4m3.cu",
-                  "mla_attention_decode_paged_b200/csrc/mla_scan_common.cuh"]
+                  "mla_attention_decode_paged_b200/csrc/mla_scan_common.cuh",
+                  "mla_attention_decode_paged_b200/csrc/mla_common.cuh",
+                  "mla_attention_decode_paged_b200/csrc/sm100_ptx.cuh"]
 
 
 def log(*a):
