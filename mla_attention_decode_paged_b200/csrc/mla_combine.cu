@@ -24,10 +24,9 @@ constexpr int kPre = 6;               // partials per thread loaded before the w
 // read by the 256 threads with one 16-byte load each.  kSplitGroups groups take the
 // splits j = group, group + kSplitGroups, ... so that kSplitGroups x kPre partials are in
 // flight before the weights are known; the group sums meet in shared memory at the end.
-// Four groups and one chunk per CTA when requests have many splits (few long requests:
-// enough CTAs, each with many partials); one group and all eight chunks when they have
-// few and there are at least 256 (request, 16-row group) pairs, so that the row weights
-// are computed once per 16 rows and the grid is one wave; two chunks for fewer pairs.
+// Launched with four groups and one chunk per CTA when requests have many splits (few
+// long requests: enough CTAs, each with many partials); requests with few splits go to
+// combine_few_kernel below.
 template <int kSplitGroups, int kChunks>
 __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups) combine_kernel(
     const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
@@ -194,6 +193,141 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     }
 }
 
+// Requests with few splits (the common case of batches of many requests): one CTA per
+// (request, 16-row group, kChunks column chunks of 64); thread t owns row t % 16 and column
+// quad t / 16 of every chunk.  The partials of two splits for all the CTA's chunks are
+// loaded at once (the first two while the lse pass runs), so a request with two splits
+// costs one round trip to memory after the weights instead of one per column chunk.
+template <int kChunks>
+__global__ void __launch_bounds__(kTileThreads, 2) combine_few_kernel(
+    const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    __shared__ float wsh[kWChunk][16];
+    __shared__ float Lsh[16], Msh[16];
+    const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
+    // launched as a programmatic dependent of the scan: nothing is read before it completes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
+    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3;
+    const int M = s_q * H;
+    const int row0 = qb * kRowsPerBlock + g * 16;
+    if (row0 >= M) return;
+    const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
+    const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
+    const int t = threadIdx.x, r16 = t & 15, cq = t >> 4;
+    const int m = row0 + r16;
+    const int c0 = blockIdx.z * kChunks;  // the CTA's first 64-column chunk
+    if (ns == 0) {
+        // a request without tokens (T_b <= 0) has no split: the planner set the status word,
+        // and its rows are written here as NaN
+        if (m < M) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+                *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * (c0 + c) + 4 * cq) =
+                    make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+            if (c0 == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
+        }
+        return;
+    }
+    if (ns == 1) return;  // written directly by the decode kernel
+    const int nqb = h->nqb;
+    // split j, chunk c: partial tile at pbase + c * 256 + j * jstride (float4); lse2 of row r
+    // at lbase[j * lstride + r]
+    const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
+                          ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + cq * 16 + r16 +
+                          (int64_t)c0 * 256;
+    const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
+    const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
+    const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
+
+    float4 x0[kChunks], x1[kChunks];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+        x0[c] = pbase[c * 256];
+        x1[c] = pbase[c * 256 + jstride];
+    }
+    {
+        // L = log2 sum_j 2^lse2_j per row: warp w takes rows 2w and 2w + 1 (one per half-warp)
+        const int lane = t & 31, r = 2 * (t >> 5) + (lane >> 4), k = lane & 15;
+        // fmaxf drops NaN, so a poisoned split (NaN lse2: a bad page or length) is tracked
+        // on its own and turns the merged row into NaN even when every split is poisoned
+        float mx = -INFINITY;
+        bool poisoned = false;
+        for (int j = k; j < ns; j += 16) {
+            const float l2 = lbase[j * lstride + r];
+            poisoned |= l2 != l2;
+            mx = fmaxf(mx, l2);
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        poisoned = ((__ballot_sync(0xffffffffu, poisoned) >> (lane & 16)) & 0xffffu) != 0;  // this row's half-warp
+        float sum = 0.f;
+        if (mx != -INFINITY)
+            for (int j = k; j < ns; j += 16) sum += fast_exp2(lbase[j * lstride + r] - mx);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (k == 0) {
+            const float nanv = __int_as_float(0x7fc00000);
+            Lsh[r] = poisoned ? nanv : mx + __log2f(sum);
+            Msh[r] = poisoned ? nanv : mx;
+        }
+    }
+    __syncthreads();
+    float4 acc[kChunks];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](const float4(&x)[kChunks], float w) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            acc[c].x += w * x[c].x; acc[c].y += w * x[c].y; acc[c].z += w * x[c].z; acc[c].w += w * x[c].w;
+        }
+    };
+#pragma unroll 1
+    for (int j0 = 0; j0 < ns; j0 += kWChunk) {
+        const int nj = min(kWChunk, ns - j0);
+        // the split weights 2^(lse2_j - L) of the 16 rows, for splits [j0, j0 + nj)
+        for (int e = t; e < nj * 16; e += kTileThreads) {
+            const int jj = e >> 4, r = e & 15;
+            const float l2 = lbase[(int64_t)(j0 + jj) * lstride + r];
+            wsh[jj][r] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - Lsh[r]);  // an empty split drops out
+        }
+        __syncthreads();
+        int jj = 0;
+        if (j0 == 0) {
+            add(x0, wsh[0][r16]);
+            add(x1, wsh[1][r16]);
+            jj = 2;
+        }
+#pragma unroll 1
+        for (; jj + 1 < nj; jj += 2) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                x0[c] = pbase[c * 256 + (j0 + jj) * jstride];
+                x1[c] = pbase[c * 256 + (j0 + jj + 1) * jstride];
+            }
+            add(x0, wsh[jj][r16]);
+            add(x1, wsh[jj + 1][r16]);
+        }
+        if (jj < nj) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) x0[c] = pbase[c * 256 + (j0 + jj) * jstride];
+            add(x0, wsh[jj][r16]);
+        }
+        __syncthreads();  // before the next weight chunk overwrites wsh
+    }
+    if (m < M) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc[c].x, acc[c].y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc[c].z, acc[c].w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * (c0 + c) + 4 * cq) = pk;
+        }
+        if (c0 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
+    }
+}
+
 mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, float* lse, cudaStream_t stream) {
     // a performance choice only (either kernel is correct for any plan): requests average
     // (B + G) / B splits under the default plan
@@ -201,7 +335,8 @@ mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, floa
     const int G = num_groups_for(sms > 0 ? sms : 1, num_row_blocks(s_q, H));
     const bool many_splits = (int64_t)B + G >= 8 * (int64_t)B;
     // with few splits a CTA takes all eight column chunks of its 16 rows when that still
-    // leaves enough CTAs (the row weights are then computed once), else two
+    // leaves enough CTAs (the row weights are then computed once, and two splits' loads
+    // for every chunk go out together), else two
     const int64_t row_groups = (int64_t)B * 4 * num_row_blocks(s_q, H);
     const int chunks = many_splits ? 1 : (row_groups >= 256 ? 8 : 2);
     cudaLaunchConfig_t cfg;
@@ -216,8 +351,8 @@ mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, floa
     cfg.numAttrs = 1;
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
     const cudaError_t e = chunks == 1   ? cudaLaunchKernelEx(&cfg, combine_kernel<4, 1>, ws, B, s_q, H, o, lse)
-                          : chunks == 8 ? cudaLaunchKernelEx(&cfg, combine_kernel<1, 8>, ws, B, s_q, H, o, lse)
-                                        : cudaLaunchKernelEx(&cfg, combine_kernel<1, 2>, ws, B, s_q, H, o, lse);
+                          : chunks == 8 ? cudaLaunchKernelEx(&cfg, combine_few_kernel<8>, ws, B, s_q, H, o, lse)
+                                        : cudaLaunchKernelEx(&cfg, combine_few_kernel<2>, ws, B, s_q, H, o, lse);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
