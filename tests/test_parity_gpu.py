@@ -128,7 +128,9 @@ def test_page_permutation_leaves_the_result_within_rounding():
                                                 (list(np.where(np.random.default_rng(2).random(5000) < 0.1, 0,
                                                                np.random.default_rng(3).integers(1, 4000, 5000))),
                                                  1, 16, 148),
-                                                ([-5, 10, 0], 2, 16, 148), ([131072] * 16, 16, 16, 148)])
+                                                ([-5, 10, 0], 2, 16, 148), ([131072] * 16, 16, 16, 148),
+                                                # the largest batch the planner's shared memory holds
+                                                (list(np.random.default_rng(4).integers(1, 200, 12000)), 1, 16, 148)])
 def test_device_plan_matches_host_restatement(lens, s_q, H, num_sms):
     import torch
     import mla_attention_decode_paged_b200 as mla
