@@ -28,7 +28,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "mla_common.cuh"
+#include "mla_decode_params.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
@@ -221,8 +221,17 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// N tile: R rounded up to 16, at most 256 (the TMEM columns of one accumulator).
-int n_tile(int R) { return std::min(256, (R + 15) / 16 * 16); }
+// N tile: R rounded up to 16, at most 256 (the TMEM columns of one accumulator), halved
+// (down to 16) while the grid of (head, M tile, N tile) CTAs has fewer CTAs than the
+// device has SMs: a CTA's time is mostly its loads' latency, so more, smaller CTAs finish
+// sooner, and the weight tiles they share come from L2.
+int n_tile(int R, int H, int m_tiles) {
+    int n = std::min(256, (R + 15) / 16 * 16);
+    const int sms = device_sm_count();
+    const int64_t want = sms > 0 ? sms : 148;
+    while (n > 16 && (int64_t)H * m_tiles * ((R + n - 1) / n) < want) n = std::max(16, (n / 2 + 15) / 16 * 16);
+    return n;
+}
 
 template <int kK>
 constexpr size_t gemm_smem_bytes(int N) {
@@ -260,7 +269,7 @@ extern "C" mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const
     if (!aligned(q_nope, 16) || !aligned(w_uk, 16) || !aligned(q_rope, 16) || !aligned(q, 16)) return MLA_ERR_INVALID_ARG;
     GemmArgs g;
     memset(&g, 0, sizeof(g));
-    g.N = n_tile(R);
+    g.N = n_tile(R, H, kDv / 128);
     // A = W_UK [H][512 d][128 k]: box of 64 k x 128 d of one head
     if (!map_3d(&g.tm_a, w_uk, 128, kDv, (uint64_t)H, 128 * 2, (uint64_t)kDv * 128 * 2, 64, 128, 1)) return MLA_ERR_CUDA;
     // X = q_nope [R][H][128 k]: box of 64 k x 1 head x N rows
@@ -281,7 +290,7 @@ extern "C" mla_status mla_project_out(const void* out, const void* w_uv, int R, 
     if (!aligned(out, 16) || !aligned(w_uv, 16) || !aligned(y, 4)) return MLA_ERR_INVALID_ARG;
     GemmArgs g;
     memset(&g, 0, sizeof(g));
-    g.N = n_tile(R);
+    g.N = n_tile(R, H, 1);
     // A = W_UV [H][512 d][128 c]: box of 64 c x 64 d of one head (MN-major atoms)
     if (!map_3d(&g.tm_a, w_uv, 128, kDv, (uint64_t)H, 128 * 2, (uint64_t)kDv * 128 * 2, 64, 64, 1)) return MLA_ERR_CUDA;
     // X = out [R][H][512 d]: box of 64 d x 1 head x N rows

@@ -28,10 +28,12 @@ def _close_bf16(got, ref):
     assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 2e-3), float((err - 2.0 ** -8 * np.abs(ref)).max())
 
 
-# R = B * s_q rows per head: 8, 256 (one full N tile), 3, 1, 64 x 128 heads (the fp8
-# workload), 15 (a ragged N tile), 320 (two N tiles)
+# R = B * s_q rows per head: 8, 256 with 16 heads (N tiles halved until the grid fills
+# the SMs), 3, 1, 64 x 128 heads (the fp8 workload), 15 (a ragged N tile), 320 with 4
+# heads (many small N tiles, the last one ragged), 256 x 64 heads (full 256-row N tiles
+# for the absorption, halved for the projection)
 @pytest.mark.parametrize("B,s_q,H", [(2, 4, 16), (16, 16, 16), (3, 1, 128), (1, 1, 1), (32, 2, 128), (3, 5, 7),
-                                     (20, 16, 4)])
+                                     (20, 16, 4), (16, 16, 64)])
 def test_absorb_and_project_match_the_oracle(B, s_q, H):
     import torch
     rng = np.random.default_rng(B * 100 + H)
