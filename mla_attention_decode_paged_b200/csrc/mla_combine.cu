@@ -18,20 +18,17 @@ constexpr int kTileThreads = 256;     // 16 rows x 16 column quads
 constexpr int kWChunk = 64;           // splits whose weights are in shared memory at once
 constexpr int kPre = 6;               // partials per thread loaded before the weights are known
 
-// One CTA per (request, 16-row group, kChunks column chunks of 64).  Within a group of
-// 256 threads, thread t owns row t % 16 and column quad t / 16 of a 16 x 64 tile; in the
-// workspace's quad-interleaved partial layout the tile of one split is 4 KB contiguous,
-// read by the 256 threads with one 16-byte load each.  kSplitGroups groups take the
-// splits j = group, group + kSplitGroups, ... so that kSplitGroups x kPre partials are in
-// flight before the weights are known; the group sums meet in shared memory at the end.
-// Launched with four groups and one chunk per CTA when requests have many splits (few
-// long requests: enough CTAs, each with many partials); requests with few splits go to
-// combine_few_kernel below.
-template <int kSplitGroups, int kChunks>
-__global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups) combine_kernel(
+// Requests with many splits (few long requests): one CTA per (request, 16-row group,
+// 64-column chunk).  Within a group of 256 threads, thread t owns row t % 16 and column
+// quad t / 16 of the 16 x 64 tile; in the workspace's quad-interleaved partial layout the
+// tile of one split is 4 KB contiguous, read by the 256 threads with one 16-byte load
+// each.  kSplitGroups groups take the splits j = group, group + kSplitGroups, ... so that
+// kSplitGroups x kPre partials are in flight before the weights are known; the group sums
+// meet in shared memory at the end.
+template <int kSplitGroups>
+__global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups) combine_many_kernel(
     const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     constexpr int kCombineThreads = kTileThreads * kSplitGroups;
-    static_assert(kSplitGroups == 1 || kChunks == 1, "split groups meet once per CTA");
     __shared__ float wsh[kWChunk][16];
     __shared__ float Lsh[16], Msh[16];
     __shared__ float4 part[kSplitGroups > 1 ? kSplitGroups - 1 : 1][kTileThreads];
@@ -39,7 +36,7 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     // launched as a programmatic dependent of the scan: nothing is read before it completes
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
-    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3;
+    const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3, c64 = blockIdx.z;
     const int M = s_q * H;
     const int row0 = qb * kRowsPerBlock + g * 16;
     if (row0 >= M) return;
@@ -52,35 +49,28 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
         // a request without tokens (T_b <= 0) has no split: the planner set the status word,
         // and its rows are written here as NaN
         if (grp == 0 && m < M) {
-#pragma unroll 1
-            for (int cc = 0; cc < kChunks; ++cc) {
-                const int c64 = blockIdx.z * kChunks + cc;
-                *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
-                    make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
-            }
-            if (blockIdx.z == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
+            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) =
+                make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+            if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = __int_as_float(0x7fc00000);
         }
         return;
     }
     if (ns == 1) return;  // written directly by the decode kernel
     const int nqb = h->nqb;
-    // split j, column chunk c64: partial tile at pbase + c64 * 256 + j * jstride (float4),
-    // lse2 of row r at lbase[j * lstride + r]
-    const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
-                          ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + cq * 16 + r16;
+    // split j: partial tile at pc + j * jstride (float4); lse2 of row r at lbase[j * lstride + r]
+    const float4* pc = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
+                       ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + (int64_t)c64 * 256 +
+                       cq * 16 + r16;
     const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
     const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
     const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
 
-    // the first chunk's partials, in flight while the weights are computed
+    // the first partials, in flight while the weights are computed
     float4 v[kPre];
-    {
-        const float4* pc = pbase + (int64_t)(blockIdx.z * kChunks) * 256;
 #pragma unroll
-        for (int u = 0; u < kPre; ++u) {
-            const int j = grp + kSplitGroups * u;
-            v[u] = j < ns ? pc[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    for (int u = 0; u < kPre; ++u) {
+        const int j = grp + kSplitGroups * u;
+        v[u] = j < ns ? pc[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
     // L = log2 sum_j 2^lse2_j per row: warp w < 8 takes rows 2w and 2w + 1 (one per half-warp)
@@ -110,86 +100,63 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
         }
     }
     __syncthreads();
-    // the split weights 2^(lse2_j - L) of the 16 rows, for splits [j0, j0 + kWChunk)
-    auto weights = [&](int j0, int nj) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int j0 = 0; j0 < ns; j0 += kWChunk) {
+        const int nj = min(kWChunk, ns - j0);
+        // the split weights 2^(lse2_j - L) of the 16 rows, for splits [j0, j0 + nj)
         for (int e = tid; e < nj * 16; e += kCombineThreads) {
             const int jj = e >> 4, r = e & 15;
             const float l2 = lbase[(int64_t)(j0 + jj) * lstride + r];
             wsh[jj][r] = (l2 == -INFINITY) ? 0.f : fast_exp2(l2 - Lsh[r]);  // an empty split drops out
         }
-    };
-    const bool one_wchunk = ns <= kWChunk;  // the weights of every split fit at once
-    if (one_wchunk) {
-        weights(0, ns);
         __syncthreads();
-    }
-#pragma unroll 1
-    for (int cc = 0; cc < kChunks; ++cc) {
-        const int c64 = blockIdx.z * kChunks + cc;
-        const float4* pc = pbase + (int64_t)c64 * 256;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j0 = 0; j0 < ns; j0 += kWChunk) {
-            const int nj = min(kWChunk, ns - j0);
-            if (!one_wchunk) {
-                weights(j0, nj);
-                __syncthreads();
-            }
-            int jj = grp;  // this group's splits within the weight chunk: grp, grp + kSplitGroups, ...
-            if (j0 == 0) {
-#pragma unroll
-                for (int u = 0; u < kPre; ++u) {
-                    const int j = grp + kSplitGroups * u;
-                    const float w = j < nj ? wsh[j][r16] : 0.f;
-                    acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
-                }
-                jj = grp + kSplitGroups * kPre;
-            }
-            for (; jj + kSplitGroups < nj; jj += 2 * kSplitGroups) {
-                float4 x[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) x[u] = pc[(j0 + jj + kSplitGroups * u) * jstride];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const float w = wsh[jj + kSplitGroups * u][r16];
-                    acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
-                }
-            }
-            for (; jj < nj; jj += kSplitGroups) {
-                const float4 x = pc[(j0 + jj) * jstride];
-                const float w = wsh[jj][r16];
-                acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
-            }
-            if (!one_wchunk) __syncthreads();
-        }
-        // the next chunk's first partials, in flight while this chunk is finished
-        if (cc + 1 < kChunks) {
-            const float4* pn = pc + 256;
+        int jj = grp;  // this group's splits within the weight chunk: grp, grp + kSplitGroups, ...
+        if (j0 == 0) {
 #pragma unroll
             for (int u = 0; u < kPre; ++u) {
                 const int j = grp + kSplitGroups * u;
-                v[u] = j < ns ? pn[j * jstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float w = j < nj ? wsh[j][r16] : 0.f;
+                acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
             }
+            jj = grp + kSplitGroups * kPre;
         }
-        if (kSplitGroups > 1) {
-            // (one chunk per CTA here: the groups' sums meet once, then the other groups leave)
-            if (grp > 0) part[grp - 1][t] = acc;
-            __syncthreads();
-            if (grp > 0) return;
+        for (; jj + kSplitGroups < nj; jj += 2 * kSplitGroups) {
+            float4 x[2];
 #pragma unroll
-            for (int k = 0; k < kSplitGroups - 1; ++k) {
-                const float4 x = part[k][t];
-                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            for (int u = 0; u < 2; ++u) x[u] = pc[(j0 + jj + kSplitGroups * u) * jstride];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float w = wsh[jj + kSplitGroups * u][r16];
+                acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
             }
         }
-        if (grp == 0 && m < M) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) = pk;
-            if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
+        for (; jj < nj; jj += kSplitGroups) {
+            const float4 x = pc[(j0 + jj) * jstride];
+            const float w = wsh[jj][r16];
+            acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
         }
+        __syncthreads();  // before the next weight chunk overwrites wsh
+    }
+    if (kSplitGroups > 1) {
+        // the groups' sums meet, then the other groups leave
+        if (grp > 0) part[grp - 1][t] = acc;
+        __syncthreads();
+        if (grp > 0) return;
+#pragma unroll
+        for (int k = 0; k < kSplitGroups - 1; ++k) {
+            const float4 x = part[k][t];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+    }
+    if (m < M) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out + ((int64_t)b * M + m) * kDv + 64 * c64 + 4 * cq) = pk;
+        if (c64 == 0 && cq == 0) lse[(int64_t)b * M + m] = (Msh[r16] == -INFINITY) ? -INFINITY : Lsh[r16] * kLn2;
     }
 }
 
@@ -350,7 +317,7 @@ mla_status launch_combine(const void* ws, int B, int s_q, int H, void* out, floa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-    const cudaError_t e = chunks == 1   ? cudaLaunchKernelEx(&cfg, combine_kernel<4, 1>, ws, B, s_q, H, o, lse)
+    const cudaError_t e = chunks == 1   ? cudaLaunchKernelEx(&cfg, combine_many_kernel<4>, ws, B, s_q, H, o, lse)
                           : chunks == 8 ? cudaLaunchKernelEx(&cfg, combine_few_kernel<8>, ws, B, s_q, H, o, lse)
                                         : cudaLaunchKernelEx(&cfg, combine_few_kernel<2>, ws, B, s_q, H, o, lse);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
