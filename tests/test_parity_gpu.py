@@ -190,6 +190,28 @@ def test_seq_len_beyond_block_table_sets_device_status():
     assert np.all(np.isfinite(lse[0].cpu().numpy()))
 
 
+@pytest.mark.parametrize("name", ["agent_spec", "fp8_batch"])
+def test_causal_length_shorter_than_the_drafts_is_reported(name):
+    """Under the draft mask a request needs at least s_q tokens (its drafts' own rows): a
+    shorter one is reported (device status) and its rows are NaN; its neighbours are exact."""
+    import torch
+    import mla_attention_decode_paged_b200 as mla
+    wl = W.make_workload(name, B=3, seq=("fixed", 700))
+    q, kv, bt, sl = pu.to_device(wl)
+    short = wl.s_q - 1  # >= 1: the request has tokens, but fewer than its drafts
+    sl_bad = torch.tensor([700, short, 700], dtype=torch.int32, device="cuda")
+    ws = mla.alloc_workspace(3, wl.s_q, wl.H)
+    out = torch.zeros((3, wl.s_q, wl.H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((3, wl.s_q, wl.H), dtype=torch.float32, device="cuda")
+    mla.plan(sl_bad, wl.s_q, wl.H, ws)
+    mla.decode(q, kv, bt, sl_bad, wl.scale, True, ws, out, lse, kv_scale=wl.kv_scale)
+    assert mla.device_status(ws) == 5
+    o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+    assert np.all(np.isnan(o[1])) and np.all(np.isnan(l[1]))
+    ref_out, ref_lse = pu.run_oracle(wl, requests=[0, 2])
+    pu.check_close(o[[0, 2]], l[[0, 2]], ref_out, ref_lse, wl.kv_dtype, what="short-request neighbours")
+
+
 def _sample_requests_and_heads(wl, segs, seed):
     """Requests the plan split and requests it held whole (the first of each, where the
     workload has them), one more seeded request, and heads {0, H-1} plus three seeded
