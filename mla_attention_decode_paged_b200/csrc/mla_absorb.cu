@@ -227,7 +227,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t
 // sooner, and the weight tiles they share come from L2.
 int n_tile(int R, int H, int m_tiles) {
     int n = std::min(256, (R + 15) / 16 * 16);
-    const int sms = device_sm_count();
+    const int sms = effective_sms();  // cached per device
     const int64_t want = sms > 0 ? sms : 148;
     while (n > 16 && (int64_t)H * m_tiles * ((R + n - 1) / n) < want) n = std::max(16, (n / 2 + 15) / 16 * 16);
     return n;
