@@ -309,6 +309,11 @@ def roofline_of(wl, scan_avg_s, traffic):
     roof["kernel"] = "mla decode split scan"
     roof["algorithmic_bytes_per_launch"] = kvb
     roof["algorithmic_flops_per_launch"] = flops
+    if roof["bound"] == "tensor" and wl.kv_dtype != W.KV_BF16:
+        # the e4m3 scan's MMAs take q and P as two e4m3 terms each (bf16 precision), so each
+        # product runs twice on the fp8 pipe: its executed FLOPs against the fp8 peak (twice
+        # the bf16 one) give the same fraction as these FLOPs against the bf16 peak
+        roof["note"] = "bf16-precision FLOPs against the bf16 peak; e4m3 MMAs run each product as two terms"
     nom_peak = NOMINAL_PEAKS["hbm_gbs"] if roof["bound"] == "hbm" else NOMINAL_PEAKS["bf16_tflops"]
     nominal = {"peak": nom_peak, "unit": roof["unit"], "frac": roof["achieved"] / nom_peak,
                "note": "B200 datasheet peak, context only"}
