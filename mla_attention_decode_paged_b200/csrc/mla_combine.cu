@@ -18,6 +18,47 @@ constexpr int kTileThreads = 256;     // 16 rows x 16 column quads
 constexpr int kWChunk = 64;           // splits whose weights are in shared memory at once
 constexpr int kPre = 6;               // partials per thread loaded before the weights are known
 
+// What a combine CTA takes from the plan: where the partials are and request b's splits.
+// It is read before the grid-dependency wait, while the scan's last CTAs still run: the
+// scan releases its dependents only after its own wait for the planner, so the plan is
+// complete when this grid starts.  One thread reads it through L2 (.cg: never a line an
+// earlier kernel left in this SM's L1; one reader, not every thread of every CTA on the
+// same lines) and hands it to the CTA in shared memory.  The partials are read only
+// after the wait.
+struct CombinePlan {
+    bool ok;
+    int nqb, s0, ns;
+    int64_t off_plse, off_po;
+};
+
+__device__ __forceinline__ CombinePlan read_combine_plan(const void* ws, int B, int s_q, int H, int b) {
+    __shared__ CombinePlan sh;
+    if (threadIdx.x == 0) {
+        const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
+        CombinePlan c;
+        const bool match = __ldcg(&h->magic) == kPlanMagic && __ldcg(&h->B) == B && __ldcg(&h->s_q) == s_q &&
+                           __ldcg(&h->H) == H;
+        c.nqb = __ldcg(&h->nqb);
+        const int max_segments = __ldcg(&h->max_segments);
+        const int64_t off_req_seg = __ldcg(reinterpret_cast<const long long*>(&h->off_req_seg));
+        c.off_plse = __ldcg(reinterpret_cast<const long long*>(&h->off_plse));
+        c.off_po = __ldcg(reinterpret_cast<const long long*>(&h->off_po));
+        c.ok = false;
+        c.s0 = c.ns = 0;
+        if (match) {
+            const int32_t* req_seg = ws_ptr<int32_t>(ws, off_req_seg);
+            const int s0 = __ldcg(req_seg + b), s1 = __ldcg(req_seg + b + 1);
+            // a plan the host accepted always passes; the check keeps every index in bounds
+            c.ok = 0 <= s0 && s0 <= s1 && s1 <= max_segments;
+            c.s0 = s0;
+            c.ns = s1 - s0;
+        }
+        sh = c;
+    }
+    __syncthreads();
+    return sh;
+}
+
 // Requests with many splits (few long requests): one CTA per (request, 16-row group,
 // 64-column chunk).  Within a group of 256 threads, thread t owns row t % 16 and column
 // quad t / 16 of the 16 x 64 tile; in the workspace's quad-interleaved partial layout the
@@ -32,16 +73,16 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
     __shared__ float wsh[kWChunk][16];
     __shared__ float Lsh[16], Msh[16];
     __shared__ float4 part[kSplitGroups > 1 ? kSplitGroups - 1 : 1][kTileThreads];
-    const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
-    // launched as a programmatic dependent of the scan: nothing is read before it completes
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
     const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3, c64 = blockIdx.z;
+    const CombinePlan cp = read_combine_plan(ws, B, s_q, H, b);
+    // launched as a programmatic dependent of the scan: no partial is read, and nothing is
+    // written, before it completes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!cp.ok) return;
     const int M = s_q * H;
     const int row0 = qb * kRowsPerBlock + g * 16;
     if (row0 >= M) return;
-    const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
-    const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
+    const int s0 = cp.s0, ns = cp.ns;
     const int tid = threadIdx.x, t = tid & (kTileThreads - 1), grp = tid / kTileThreads;
     const int r16 = t & 15, cq = t >> 4;
     const int m = row0 + r16;
@@ -56,13 +97,13 @@ __global__ void __launch_bounds__(kTileThreads * kSplitGroups, 4 / kSplitGroups)
         return;
     }
     if (ns == 1) return;  // written directly by the decode kernel
-    const int nqb = h->nqb;
+    const int nqb = cp.nqb;
     // split j: partial tile at pc + j * jstride (float4); lse2 of row r at lbase[j * lstride + r]
-    const float4* pc = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
+    const float4* pc = reinterpret_cast<const float4*>(ws_ptr<float>(ws, cp.off_po)) +
                        ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + (int64_t)c64 * 256 +
                        cq * 16 + r16;
     const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
-    const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
+    const float* lbase = ws_ptr<float>(ws, cp.off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
     const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
 
     // the first partials, in flight while the weights are computed
@@ -170,16 +211,16 @@ __global__ void __launch_bounds__(kTileThreads, 2) combine_few_kernel(
     const void* __restrict__ ws, int B, int s_q, int H, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     __shared__ float wsh[kWChunk][16];
     __shared__ float Lsh[16], Msh[16];
-    const PlanHeader* h = reinterpret_cast<const PlanHeader*>(ws);
-    // launched as a programmatic dependent of the scan: nothing is read before it completes
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (h->magic != kPlanMagic || h->B != B || h->s_q != s_q || h->H != H) return;
     const int b = blockIdx.x, qb = blockIdx.y >> 2, g = blockIdx.y & 3;
+    const CombinePlan cp = read_combine_plan(ws, B, s_q, H, b);
+    // launched as a programmatic dependent of the scan: no partial is read, and nothing is
+    // written, before it completes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!cp.ok) return;
     const int M = s_q * H;
     const int row0 = qb * kRowsPerBlock + g * 16;
     if (row0 >= M) return;
-    const int32_t* req_seg = ws_ptr<int32_t>(ws, h->off_req_seg);
-    const int s0 = req_seg[b], ns = req_seg[b + 1] - s0;
+    const int s0 = cp.s0, ns = cp.ns;
     const int t = threadIdx.x, r16 = t & 15, cq = t >> 4;
     const int m = row0 + r16;
     const int c0 = blockIdx.z * kChunks;  // the CTA's first 64-column chunk
@@ -196,14 +237,14 @@ __global__ void __launch_bounds__(kTileThreads, 2) combine_few_kernel(
         return;
     }
     if (ns == 1) return;  // written directly by the decode kernel
-    const int nqb = h->nqb;
+    const int nqb = cp.nqb;
     // split j, chunk c: partial tile at pbase + c * 256 + j * jstride (float4); lse2 of row r
     // at lbase[j * lstride + r]
-    const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, h->off_po)) +
+    const float4* pbase = reinterpret_cast<const float4*>(ws_ptr<float>(ws, cp.off_po)) +
                           ((int64_t)s0 * nqb + qb) * (kRowsPerBlock * kDv / 4) + g * 2048 + cq * 16 + r16 +
                           (int64_t)c0 * 256;
     const int64_t jstride = (int64_t)nqb * (kRowsPerBlock * kDv / 4);
-    const float* lbase = ws_ptr<float>(ws, h->off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
+    const float* lbase = ws_ptr<float>(ws, cp.off_plse) + ((int64_t)s0 * nqb + qb) * kRowsPerBlock + g * 16;
     const int64_t lstride = (int64_t)nqb * kRowsPerBlock;
 
     float4 x0[kChunks], x1[kChunks];

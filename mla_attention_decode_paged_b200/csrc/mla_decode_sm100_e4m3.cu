@@ -106,8 +106,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
     const DecodeParams& p = args.p;
     PlanHeader* h = reinterpret_cast<PlanHeader*>(p.ws);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // the combine may start its prologue now; it waits for this grid before reading
-    ptx::griddep_launch_dependents();
 
     // prologue that reads no global memory, ahead of the wait for the grid before this one
     Ctx c;
@@ -140,6 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_e4m3_kernel(const __grid_c
 
     // the plan (and every earlier write) must be complete before the header is read
     ptx::griddep_wait();
+    // Only now may the combine launch: it reads the plan before its own wait for this grid
+    // (the plan is complete once the wait above returns), the partials after it.
+    ptx::griddep_launch_dependents();
     // The header and this group's head record are read together: the head table sits at a
     // fixed offset, and every workspace the host accepts holds it for any group launched.
     const int nqb = num_row_blocks(p.s_q, p.H);

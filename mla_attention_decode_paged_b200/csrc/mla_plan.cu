@@ -224,10 +224,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         h->off_plse = L.off_plse;
         h->off_po = L.off_po;
         h->total_bytes = L.total;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
+        // every reader of the plan starts after this grid has completed (stream order, or
+        // a programmatic dependent's grid-dependency wait): no fence orders the magic last
         h->magic = kPlanMagic;
     }
 }
