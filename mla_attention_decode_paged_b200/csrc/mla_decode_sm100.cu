@@ -12,18 +12,26 @@
 // Tensor memory (128 lanes x 512 columns) with 64-row MMAs, whose rows occupy 16 lanes
 // of each 32-lane subpartition:
 //   lanes at offset 0  : O, the 64 x 512 fp32 output accumulator (all 512 columns)
-//   lanes at offset 16 : q (64 x 576 bf16, 288 columns, loaded once per split) and two
-//                        64-column score buffers.
+//   lanes at offset 16 : q's latent part (64 x 512 bf16, 256 columns, loaded once per
+//                        split), two 64-column buffers for the first half of each page's
+//                        scores and two for the second half.
+// q's rope part (64 x 64 bf16, 8 KB) sits in shared memory, in the epilogue's staging tile
+// (which the epilogue needs only after the split's last MMA), as the A operand of the
+// four rope K-steps.
 // Per page:
 //   TMA (producer warp): the page's 64 rows x 576 columns as nine 64-column boxes with
 //       128-byte swizzle (one 72 KB stage; three stages).
-//   MMA (one thread): S = q . K^T with q read from TMEM (M=64 N=64 K=16, 36 K-steps),
-//       then O += P . V with P (bf16) and V (the same page, read MN-major) from shared
-//       memory (M=64 N=256 K=16, twice, 4 K-steps each).  P is written over the page's
-//       rope chunk, which only the score MMAs read: every stage carries its own P, and
-//       the softmax of a page never waits for the previous page's PV.
-//   softmax (4 warps, 16 rows each, two threads per row with 32 scores each): base-2
-//       online softmax with the causal draft mask; the running max is only raised (and
+//   MMA (two threads): S = q . K^T (M=64 N=64 K=16, 36 K-steps), its first 18 K-steps
+//       issued by one thread (warp 1) and its last 18 by another (warp 6) into a second
+//       accumulator: one thread issuing a 64-row MMA takes about as long as the tensor core
+//       takes to run it, so one issuer alone leaves the tensor core short of work.  q comes
+//       from TMEM, except in the four rope K-steps.  Warp 1 also issues O += P . V with P
+//       (bf16) and V (the same page, read MN-major) from shared memory (M=64 N=256 K=16,
+//       twice, 4 K-steps each).  P is written over the page's rope chunk, which only the
+//       score MMAs read: every stage carries its own P, and the softmax of a page never
+//       waits for the previous page's PV.
+//   softmax (4 warps, 16 rows each, two threads per row with 32 scores each): adds the
+//       two halves of the scores, base-2 online softmax with the causal draft mask; the running max is only raised (and
 //       O rescaled) when a score exceeds it by more than 8, so P <= 256.
 //   epilogue: O / l -> bf16 out (a request the split holds whole) or an fp32 partial and
 //       its base-2 lse (split request; merged by the combine kernel).
@@ -40,6 +48,9 @@ namespace {
 using namespace scan;
 
 constexpr int kStages = 3;
+// warp 0 TMA, warp 1 score chain (first half) and PV, warps 2-5 softmax / epilogue, warp 6
+// score chain (second half)
+constexpr int kThreadsBf16 = kThreads + 32;
 constexpr uint32_t kChunk = kTok * 128;              // 64 tokens x 64 columns bf16, 128B-swizzled
 constexpr uint32_t kStageBytes = 9 * kChunk;         // 8 latent chunks + 1 rope chunk: 72 KB
 constexpr uint32_t kOffKv = 0;
@@ -52,33 +63,48 @@ static_assert(kSmemBytes <= (uint32_t)kMaxSmem, "dynamic shared memory limit per
 
 enum : int {
     B_KV_FULL0 = 0, B_KV_EMPTY0 = B_KV_FULL0 + kStages, B_Q_FULL = B_KV_EMPTY0 + kStages, B_S_FULL0,
-    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_DRAIN = B_PV_DONE0 + 2, B_COUNT
+    B_P_READY0 = B_S_FULL0 + 2, B_PV_DONE0 = B_P_READY0 + 2, B_DRAIN = B_PV_DONE0 + 2,
+    B_SB_FULL0, B_SB_FREE0 = B_SB_FULL0 + 2, B_DRAIN_B = B_SB_FREE0 + 2, B_COUNT
 };
 constexpr uint32_t kOffTmemHolder = kOffBar + 8 * B_COUNT;
 constexpr uint32_t kOffAbort = kOffTmemHolder + 4;
 static_assert(kOffAbort + 4 <= kOffBar + 256, "barrier area");
 
-constexpr uint32_t kColQ = 0;            // q: 288 columns (bf16 pairs)
-constexpr uint32_t kColS = 288;          // scores: 2 x 64 columns
+constexpr uint32_t kColQ = 0;            // q, dims 0-511: 256 columns (bf16 pairs)
+constexpr uint32_t kColS = 256;          // scores, K-steps [0, kHalfSteps): 2 x 64 columns
+constexpr uint32_t kColSB = 384;         // scores, K-steps [kHalfSteps, 36): 2 x 64 columns
+constexpr int kHalfSteps = 18;
+constexpr int kRopeStep = 32;            // K-steps 32-35 read q's rope part from shared memory
+static_assert(kHalfSteps <= kRopeStep, "the first issuer reads q from TMEM only");
+static_assert(kRows * 128 == 4 * kEpiWarpBytes, "q's rope part fills the epilogue staging tile");
 constexpr float kRescaleThreshold = 8.0f;
 
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRows, kTok, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kRows, 256, 0, 1);
 
-// Twelve score K-steps starting at K0 (of 36): q from TMEM, the page from shared memory.
-// K0 is a template constant so that every descriptor offset is an immediate.
-template <int K0>
-__device__ __forceinline__ void issue_s_chunk(uint32_t d, uint32_t a0, uint64_t b0) {
+// Score K-steps [K0, K0 + NK) (of 36) into accumulator d, the first of them overwriting it:
+// q from TMEM, the page from shared memory.  K0 is a template constant so that every
+// descriptor offset is an immediate.
+template <int K0, int NK>
+__device__ __forceinline__ void issue_s_steps(uint32_t d, uint32_t a0, uint64_t b0) {
 #pragma unroll
-    for (int k = 0; k < 12; ++k) {
+    for (int k = 0; k < NK; ++k) {
         constexpr int kChunkUnits = kChunk >> 4;
         const int ks = K0 + k;
         ptx::mma_ts(d, a0 + 8u * ks, b0 + (uint64_t)((ks >> 2) * kChunkUnits + (ks & 3) * 2), kIdescS,
-                    ks ? 1u : 0u);
+                    k ? 1u : 0u);
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_constant__ Args args) {
+// The four rope K-steps (32-35), accumulating into d: A = q's rope part from shared memory
+// (K-major, 128-byte swizzle, like P), B = the page's rope chunk.
+__device__ __forceinline__ void issue_s_rope(uint32_t d, uint64_t aq, uint64_t b0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        ptx::mma_ss(d, aq + (uint64_t)(k * 2), b0 + (uint64_t)(8 * (kChunk >> 4) + k * 2), kIdescS, 1u);
+}
+
+__global__ void __launch_bounds__(kThreadsBf16, 1) decode_sm100_kernel(const __grid_constant__ Args args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
@@ -104,6 +130,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
             ptx::mbar_init(c.bar(B_PV_DONE0 + s), 1);
         }
         ptx::mbar_init(c.bar(B_DRAIN), 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(c.bar(B_SB_FULL0 + s), 1);
+            ptx::mbar_init(c.bar(B_SB_FREE0 + s), 128);
+        }
+        ptx::mbar_init(c.bar(B_DRAIN_B), 1);
         ptx::fence_mbar_init_cluster();
     }
     if (warp == 0 && lane == 0) ptx::prefetch_tmap(&args.tm_kv);
@@ -190,10 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // An event loop: the score MMAs of the next page and the PV MMAs of the oldest
-        // page whose P is ready are issued in whichever order their inputs arrive.  The
-        // tensor core runs them in issue order.  Barriers are polled with test_wait, which
-        // never suspends the thread.
+        // An event loop: the first half of the next page's score MMAs and the PV MMAs of the
+        // oldest page whose P is ready are issued in whichever order their inputs arrive.
+        // Barriers are polled with test_wait, which never suspends the thread.
         if (lane == 0) {
             int it = 0, nseg = 0;
             bool ok = true;
@@ -209,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
                 while (npv < n) {
                     bool progressed = false;
                     // S(ns) reuses the score buffer of page ns-2, whose PV must be issued first.
-                    // A score chain is issued whole: PV MMAs placed between its K-steps (another
-                    // accumulator) slow the chain down far more than they gain.
+                    // The chain's half is issued whole: PV MMAs placed between its K-steps (another
+                    // accumulator) slow it down far more than they gain.
                     if (ns < n && ns <= npv + 1) {
                         const int its = it + ns, st = its % kStages;
                         if (ptx::mbar_test_wait(c.bar(B_KV_FULL0 + st), (its / kStages) & 1)) {
@@ -221,9 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
                                                                ptx::kSwizzle128);
                             const uint32_t d = tmem + kLaneHi + kColS + 64u * (its & 1);
                             const uint32_t a0 = tmem + kLaneHi + kColQ;
-                            issue_s_chunk<0>(d, a0, b0);
-                            issue_s_chunk<12>(d, a0, b0);
-                            issue_s_chunk<24>(d, a0, b0);
+                            issue_s_steps<0, kHalfSteps>(d, a0, b0);
                             ptx::mma_commit(c.bar(B_S_FULL0 + (its & 1)));
                             ++ns;
                             progressed = true;
@@ -264,6 +292,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
             ptx::mma_commit(c.bar(B_DRAIN));
             drain_wait(c.bar(B_DRAIN), 0);
         }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ second score issuer
+        const uint64_t aq = ptx::smem_desc(sbase + kOffEpi, 16, 1024, ptx::kSwizzle128);
+        // K-steps [kHalfSteps, 36) of every page's score chain into the second-half buffers.
+        // It walks the same pages as the first issuer; a page's half is issued once its
+        // stage is full and the softmax warps have loaded the half of the page two before
+        // (SB_FREE, the same buffer), so no SB_FULL phase runs ahead of its waiters.
+        if (lane == 0) {
+            int it = 0, nseg = 0;
+            bool ok = true;
+            for (int si = seg_lo; si < seg_hi && ok; ++si) {
+                const Segment S = si == seg_lo ? gh.first : segs[si];
+                const int T = p.seq_lens[S.b];
+                if (!request_ok(p, T)) continue;
+                if (!wait_bar(c, c.bar(B_Q_FULL), nseg & 1)) break;
+                ptx::tc_fence_after();
+                const int n = S.tile_end - S.tile_begin;
+                for (int j = 0; j < n; ++j) {
+                    const int its = it + j, st = its % kStages;
+                    if ((its >= 2 && !wait_bar(c, c.bar(B_SB_FREE0 + (its & 1)), ((its - 2) >> 1) & 1)) ||
+                        !wait_bar(c, c.bar(B_KV_FULL0 + st), (its / kStages) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint64_t b0 = ptx::smem_desc(sbase + kOffKv + st * kStageBytes, 16, 1024, ptx::kSwizzle128);
+                    const uint32_t d = tmem + kLaneHi + kColSB + 64u * (its & 1);
+                    issue_s_steps<kHalfSteps, kRopeStep - kHalfSteps>(d, tmem + kLaneHi + kColQ, b0);
+                    issue_s_rope(d, aq, b0);
+                    ptx::mma_commit(c.bar(B_SB_FULL0 + (its & 1)));
+                }
+                it += n;
+                ++nseg;
+            }
+            ptx::mma_commit(c.bar(B_DRAIN_B));
+            drain_wait(c.bar(B_DRAIN_B), 0);
+        }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         RowSlot r;
@@ -289,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         for (int si = seg_lo; si < seg_hi; ++si) {
             const Segment S = si == seg_lo ? gh.first : segs[si];
             const int T = p.seq_lens[S.b];
-            // q rows of this block into TMEM: 9 x (16 columns per half) = 576 bf16 per row.
+            // q rows of this block: dims 0-511 into TMEM (8 x 16 columns per half), the rope
+            // part into shared memory.
             // The loads are all issued before the first is used, beside the length's read: at a
             // split's start the memory system is full of the first pages' loads, and every
             // dependent round trip here delays the first score MMA.
@@ -308,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
             if (*c.abort) break;
             {
 #pragma unroll
-                for (int k = 0; k < 9; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     uint32_t v[16];
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
@@ -319,6 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
                     }
                     ptx::tmem_st16x16<16>(t_hi + kColQ + 32u * k, v);
                 }
+                // the rope part: row `row`, dims [512 + 32 half, +32) as four 16-byte pieces of
+                // the row's 128 bytes, 128-byte swizzle; the rows of this warp's quadrant are its
+                // own epilogue staging tile, which its previous epilogue has finished with
+                uint8_t* qrow = smem + kOffEpi + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    *reinterpret_cast<uint4*>(qrow + (((4 * half + w) ^ (row & 7)) << 4)) = x[8][w];
+                ptx::fence_proxy_async_smem();
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(c.bar(B_Q_FULL));
@@ -334,22 +408,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
                 const int tile = S.tile_begin + jj;
                 const int32_t page = p.block_table[(int64_t)S.b * p.max_pages + tile];
                 badpage |= !(page >= 0 && page < p.num_pages);
-                alive = wait_bar(c, c.bar(B_S_FULL0 + (it & 1)), (it >> 1) & 1);
+                alive = wait_bar(c, c.bar(B_S_FULL0 + (it & 1)), (it >> 1) & 1) &&
+                        wait_bar(c, c.bar(B_SB_FULL0 + (it & 1)), (it >> 1) & 1);
                 if (__any_sync(0xffffffffu, !alive)) { alive = false; break; }
                 ptx::tc_fence_after();
-                uint32_t sr[32];
+                uint32_t sr[32], sr2[32];
                 ptx::tmem_ld16x32<32>(t_hi + kColS + 64u * (it & 1), sr);
+                ptx::tmem_ld16x32<32>(t_hi + kColSB + 64u * (it & 1), sr2);
                 ptx::tmem_wait_ld();
+                // this second-half buffer may take the half of the page two ahead
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(c.bar(B_SB_FREE0 + (it & 1)));
                 float s[32];
                 const int tok0 = tile * kPage + 32 * half;
                 if (tile * kPage + kPage <= full_end) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(sr[k]) * sc;
+                    for (int k = 0; k < 32; ++k) s[k] = (__uint_as_float(sr[k]) + __uint_as_float(sr2[k])) * sc;
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
                         const int t = tok0 + k;
-                        s[k] = (t < T && t <= last_t) ? __uint_as_float(sr[k]) * sc : -INFINITY;
+                        s[k] = (t < T && t <= last_t) ? (__uint_as_float(sr[k]) + __uint_as_float(sr2[k])) * sc
+                                                      : -INFINITY;
                     }
                 }
                 float mx[8];
@@ -425,7 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
             const float nanv = __int_as_float(0x7fc00000);
             const float inv = badpage ? nanv : (l > 0.f ? p.out_scale / l : 0.f);
             const float lse2 = badpage ? nanv : (l > 0.f ? m_run + __log2f(l) : -INFINITY);
-            store_split(p, S, si, r, t_lo, smem + kOffEpi + (warp - 2) * kEpiWarpBytes, inv, lse2, po, plse);
+            // the staging tile of this warp holds its quadrant's rows of q's rope part, which the
+            // split's score MMAs (all complete: the last PV is) no longer read
+            store_split(p, S, si, r, t_lo, smem + kOffEpi + r.quad * kEpiWarpBytes, inv, lse2, po, plse);
             // the next split's q overwrites TMEM only after this epilogue's reads (same threads)
             ptx::tc_fence_before();
         }
@@ -504,7 +586,7 @@ mla_status launch_bf16(const DecodeParams& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(ctas);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kThreadsBf16);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -557,7 +639,7 @@ int sm100_cta_slots() {
     if (dev < 64 && cached[dev] > 0) return cached[dev];
     if (!smem_attribute_set(dev)) return -1;
     int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_sm100_kernel, kThreads, kSmemBytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_sm100_kernel, kThreadsBf16, kSmemBytes) !=
             cudaSuccess ||
         per_sm <= 0)
         return -1;

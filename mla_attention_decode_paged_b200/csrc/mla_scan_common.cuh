@@ -4,10 +4,11 @@
 // the scan must poison, and the epilogue that turns the TMEM accumulator into the bf16
 // output or an fp32 split partial.
 //
-// Both kernels use the same CTA: 192 threads (warp 0 TMA producer, warp 1 MMA issuer,
-// warps 2-5 softmax and epilogue), one block of 64 folded query rows, 64-row tcgen05
-// MMAs whose rows occupy 16 lanes of each 32-lane TMEM subpartition: O (64 x 512 fp32)
-// in the lanes at offset 0, q and the scores in the lanes at offset 16.
+// Both kernels use the same CTA roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2-5
+// softmax and epilogue (192 threads; the bf16 scan adds warp 6, a second score issuer),
+// one block of 64 folded query rows, 64-row tcgen05 MMAs whose rows occupy 16 lanes of
+// each 32-lane TMEM subpartition: O (64 x 512 fp32) in the lanes at offset 0, q and the
+// scores in the lanes at offset 16.
 #pragma once
 
 #include <cudaTypedefs.h>
